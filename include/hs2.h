@@ -1,0 +1,197 @@
+/*
+ * hs2.h - C ABI of the HySparse2 hybrid-block attention path on NVIDIA B200 (sm_100a).
+ *
+ * One Hybrid Block = one Full Attention layer followed by several Sparse
+ * Attention layers.  The full-attention layer reads the whole KV cache and also
+ * decides which tokens matter; the sparse layers reuse that cache and that
+ * token selection (KV Reuse).  Sources, by page title and section:
+ *   [HT]  "Xiaomi Unveils HySparse2 for Faster Long-Context AI",
+ *         sections "Two-Level KV Sharing" and "Token-Level Selection and
+ *         Unified Local Access".
+ *   [OH]  "Xiaomi Releases HySparse2, Targeting Long-Horizon Reasoning for
+ *         Agents", section "From Hybrid SWA to HySparse2, Xiaomi Continues to
+ *         Refine the Attention Structure".
+ *   [BB]  "Xiaomi discloses MiMo-V3 plans to adopt HySparse2 architecture",
+ *         section "Article".
+ *   [LF]  "MiMo-V3 Architecture Revealed: HySparse2 ...", section
+ *         "Token-Level Sparse Selection and Deployment Optimization".
+ *
+ * The four calls of one decode or chunk step, in order:
+ *   hs2_full_attn_scores  full attention of the query tokens + per-key scores
+ *   hs2_topk_select       token-level top-k outside the window, plus the window
+ *   hs2_sparse_attn       one sparse layer over the selected rows (call once
+ *                         per reuse layer, each with its own queries)
+ *   hs2_block_select      (comparison path) first-generation block selection
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Layout.  Token-major and packed over the batch.  For B sequences with query
+ *   lengths Tq_b and cache lengths N_b:
+ *     Q, O        [total_q,  Hq,  D]   total_q  = sum_b Tq_b
+ *     K, V        [total_kv, Hkv, D]   total_kv = sum_b N_b
+ *   contiguous, row-major, element type ``dtype`` (HS2_BF16 or HS2_F32; all
+ *   of Q, K, V and O share it).  Query head h reads KV head h / (Hq / Hkv).
+ *   D must be 128.  Query row i (0-based) of sequence b sits at absolute
+ *   position t = N_b - Tq_b + i and sees cache positions 0..t (causal).  The
+ *   query's own key is already in the cache.
+ * Rows.  A selection row is one (query row, KV head) pair:
+ *   row = query_row * Hkv + kv_head, R = total_q * Hkv rows.
+ * Scores.  float32 [R, score_stride]: entry j of a row is the score of cache
+ *   position j of that row's sequence.  Only entries 0..t are defined.
+ * Indices.  int32 positions relative to the start of the row's sequence.
+ * Pointers.  Every tensor pointer is a DEVICE pointer, 16-byte aligned.  The
+ *   offsets in hs2_problem are device pointers too; their host copies
+ *   total_q / total_kv / max_q_len / max_kv_len must agree with them.
+ * Ownership.  The caller owns every buffer, including the workspace.  The
+ *   library allocates no memory, never synchronises (except
+ *   hs2_get_last_device_error) and launches only on ``stream``
+ *   (a cudaStream_t; NULL is the legacy default stream).  Calls may be captured
+ *   in a CUDA graph.  Calls that use the same workspace must not overlap.
+ * Workspace.  Query the size with the matching *_workspace_size call; pass at
+ *   least that many bytes, 256-byte aligned.  Its contents on entry do not
+ *   matter; on return they are unspecified.
+ * Errors.  Arguments are checked on the host before any launch; a failed check
+ *   returns an error code and launches nothing.  A CUDA launch failure returns
+ *   HS2_ERR_CUDA.  Conditions only the device can see (offsets that disagree
+ *   with the host totals, an index outside 0..t) are recorded in a device error
+ *   word, the offending work is skipped, and hs2_get_last_device_error reports
+ *   them.  Inputs must be finite; NaN / Inf give unspecified results.
+ */
+#ifndef HS2_H
+#define HS2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HS2_OK = 0,
+  HS2_ERR_INVALID_ARG = -1,  /* bad pointer, size, stride or shape                */
+  HS2_ERR_UNSUPPORTED = -2,  /* valid but not built (D != 128, group size, ...)     */
+  HS2_ERR_WORKSPACE = -3,    /* workspace missing, too small or misaligned          */
+  HS2_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed          */
+  HS2_ERR_TIMEOUT = -5,      /* a bounded device-side wait ran out                   */
+  HS2_ERR_DEVICE_INPUT = -6  /* the device found inputs that break the contract      */
+} hs2_status;
+
+typedef enum { HS2_F32 = 0, HS2_BF16 = 1 } hs2_dtype;
+
+/* Shapes of one batch.  All fields are read on the host; the two offset
+ * arrays are device pointers read by the kernels. */
+typedef struct {
+  int32_t B;                 /* sequences in the batch, >= 1                        */
+  int32_t Hq;                /* query heads                                         */
+  int32_t Hkv;               /* KV heads; Hq % Hkv == 0                             */
+  int32_t D;                 /* head dimension; must be 128                         */
+  int32_t dtype;             /* hs2_dtype of Q, K, V, O                             */
+  int32_t reserved;          /* must be 0                                           */
+  const int64_t* q_offsets;  /* device [B+1], prefix sums of Tq_b, q_offsets[0] = 0  */
+  const int64_t* kv_offsets; /* device [B+1], prefix sums of N_b,  kv_offsets[0] = 0 */
+  int64_t total_q;           /* = q_offsets[B]                                      */
+  int64_t total_kv;          /* = kv_offsets[B]                                     */
+  int64_t max_q_len;         /* >= every Tq_b; 1 selects the decode kernels          */
+  int64_t max_kv_len;        /* >= every N_b; every N_b must be >= Tq_b             */
+  float scale;               /* softmax scale applied to q.k, e.g. 1/sqrt(D)        */
+} hs2_problem;
+
+/* ---------------------------------------------------------------------------
+ * hs2_full_attn_scores - the Full Attention layer of a Hybrid Block, which
+ * both produces the attention output over the whole KV cache and decides
+ * which tokens are important ([OH]; [HT] "Two-Level KV Sharing", KV Reuse).
+ *
+ * For every query row (position t) and query head h:
+ *   x_j = scale * q_h . k_{g(h), j}   for j = 0..t
+ *   P_hj = exp(x_j - max x) / sum_j exp(x_j - max x),   O_h = sum_j P_hj v_j
+ * and, for every KV head g, the selection score of position j
+ *   scores[row(query, g)][j] = sum over the G query heads h of group g of P_hj
+ * (the pages do not define the score; this sum of the group's probabilities is
+ * the reading this library implements).  Scores are float32; O has ``dtype``.
+ *
+ * Q [total_q, Hq, D], K / V [total_kv, Hkv, D]: inputs.  O [total_q, Hq, D]:
+ * output.  scores [R, score_stride] float32: output, score_stride >= max_kv_len.
+ * Decode (max_q_len == 1) streams the cache once; chunks (max_q_len > 1) make a
+ * second pass over K to write the scores.
+ * Returns HS2_OK, or INVALID_ARG / UNSUPPORTED / WORKSPACE / CUDA.
+ */
+hs2_status hs2_full_attn_workspace_size(const hs2_problem* p, size_t* bytes);
+hs2_status hs2_full_attn_scores(const hs2_problem* p, const void* Q, const void* K,
+                                const void* V, void* O, float* scores, int64_t score_stride,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * hs2_topk_select - token-level selection ([HT] "Token-Level Selection and
+ * Unified Local Access"; [BB]; [LF]).  For each row with query position t:
+ *   window     = positions [max(0, t-window+1), t]          (always kept)
+ *   candidates = positions [0, t-window]                    (outside the window)
+ *   global     = the k candidates with the highest score; equal scores are
+ *                ordered by lower position (deterministic, independent of
+ *                the launch shape); all candidates if there are at most k.
+ * idx [R, k+window] int32: output, global positions ascending, then the window
+ * ascending, then -1 padding.  count [R] int32: output, number of valid
+ * entries = min(#candidates, k) + min(t+1, window).
+ * Scores are compared as float32 values (-0.0 == +0.0).  1 <= k, window.
+ * Results are bit-identical to a full sort by (score desc, position asc).
+ */
+hs2_status hs2_topk_workspace_size(const hs2_problem* p, int32_t k, int32_t window,
+                                   size_t* bytes);
+hs2_status hs2_topk_select(const hs2_problem* p, const float* scores, int64_t score_stride,
+                           int32_t k, int32_t window, int32_t* idx, int32_t* count,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * hs2_block_select - the first-generation HySparse block-level selection, kept
+ * as a comparison path ([BB]: groups of 64 tokens kept whole).  Candidates as
+ * in hs2_topk_select.  Block b covers positions [block*b, block*b+block-1];
+ * its score is the maximum score of its candidate positions; blocks without a
+ * candidate are not eligible.  The n_blocks best blocks (equal scores: lower
+ * block index first) contribute all their candidate positions, ascending,
+ * followed by the window.
+ * idx [R, n_blocks*block + window] int32 (-1 padded), count [R] int32.
+ */
+hs2_status hs2_block_select_workspace_size(const hs2_problem* p, int32_t n_blocks,
+                                           int32_t block, int32_t window, size_t* bytes);
+hs2_status hs2_block_select(const hs2_problem* p, const float* scores, int64_t score_stride,
+                            int32_t n_blocks, int32_t block, int32_t window, int32_t* idx,
+                            int32_t* count, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------
+ * hs2_sparse_attn - one Sparse Attention layer that reuses the full-attention
+ * layer's KV cache and index set ([HT] "Two-Level KV Sharing", KV Reuse, and
+ * "Token-Level Selection and Unified Local Access": local and global tokens in
+ * one sparse computation over the shared cache).  For every query row and
+ * query head h of KV group g, with I = idx[row(query, g)][0 .. count-1]:
+ *   O_l,h = sum_{j in I} softmax_I(scale * q_l,h . k_{g,j}) v_{g,j}
+ * Q_l [total_q, Hq, D]: this layer's queries.  K / V: the same cache as the
+ * full-attention call.  idx [R, idx_stride], count [R]: from a select call
+ * (0 <= count <= idx_stride).  O_l [total_q, Hq, D]: output.  A row with
+ * count 0 gives O = 0.  An index outside 0..t is recorded as
+ * HS2_ERR_DEVICE_INPUT and skipped.
+ */
+hs2_status hs2_sparse_attn_workspace_size(const hs2_problem* p, int32_t idx_stride,
+                                          size_t* bytes);
+hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K,
+                           const void* V, const int32_t* idx, const int32_t* count,
+                           int32_t idx_stride, void* O_l, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Device error word.  Synchronises ``stream``, returns the first error any
+ * kernel of this library recorded on the current device since the last call
+ * (HS2_OK if none) and clears it.  HS2_ERR_CUDA if the synchronisation fails.
+ */
+hs2_status hs2_get_last_device_error(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* hs2_status_string(hs2_status s);
+
+/* Library version, (major << 16) | minor. */
+int32_t hs2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HS2_H */

@@ -1,0 +1,402 @@
+// decode_attn.cuh - Full Attention layer of a Hybrid Block for decode (one query
+// token per sequence), which also emits the per-key selection scores.
+//
+// Source: "Xiaomi Releases HySparse2, Targeting Long-Horizon Reasoning for
+// Agents", section "From Hybrid SWA to HySparse2 ..." (the full-attention layer
+// builds the KV cache and decides which tokens are important) and "Xiaomi
+// Unveils HySparse2 for Faster Long-Context AI", section "Two-Level KV Sharing".
+//
+// Three launches:
+//   1. k_decode_bf16 / k_decode_f32: split-context pass.  The packed key space
+//      of every KV head is cut into P balanced ranges, one per CTA, regardless
+//      of sequence boundaries (ragged batches stay balanced).  A CTA streams its
+//      K/V rows once, writes the scaled logits x_hj of its keys, and keeps an
+//      online-softmax partial (m, l, O) per warp and per sequence piece.
+//   2. k_decode_combine: merges the partials of each (sequence, head) into the
+//      output O and the final softmax statistics (m_h, l_h).
+//   3. k_finalize_scores: s_g[j] = sum_{h in g} exp(x_hj - m_h) / l_h.
+// The per-head logits must be stored because the score needs each head's final
+// statistics, which are only known after the whole cache has been read; storing
+// them (32 B per key and KV head at G = 8) is far cheaper than reading K twice.
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace hs2 {
+
+constexpr int kDecTile = 64;        // keys per pipeline stage
+constexpr int kDecWarps = 4;        // consumer warps, 16 keys of each tile each
+constexpr int kDecStageBytes = 4 * 8192;  // K and V, two 64-column swizzled halves each
+
+struct DecodeArgs {
+  const void* Q;          // [total_q, Hq, D]
+  const void* K;          // [total_kv, Hkv, D] (CUDA-core path)
+  const void* V;
+  const int64_t* qoff;
+  const int64_t* kvoff;
+  int B, Hq, Hkv, G, P;   // P: CTAs per KV head
+  int64_t total_q, total_kv;
+  float scale;
+  float* logits;          // [total_kv, Hq]
+  float* pm;              // [(P+B), Hkv, kDecWarps, G]
+  float* pl;
+  float* po;              // [(P+B), Hkv, kDecWarps, G, D]
+  int* err;
+};
+
+// Walks the pieces (sequence b, key range [s, e)) of CTA p's key range; for
+// each piece whose sequence has a query row, calls f(b, s, e, q0).
+template <typename F>
+__device__ __forceinline__ void for_each_piece(const DecodeArgs& a, int p, F f) {
+  const int64_t W = a.total_kv;
+  const int64_t lo = split_lo(W, a.P, p), hi = split_lo(W, a.P, p + 1);
+  if (lo >= hi) return;
+  for (int b = last_le(a.kvoff, a.B, lo); b < a.B; ++b) {
+    const int64_t kb = __ldg(a.kvoff + b), ke = __ldg(a.kvoff + b + 1);
+    if (kb >= hi) break;
+    const int64_t s = kb > lo ? kb : lo, e = ke < hi ? ke : hi;
+    if (s >= e) continue;
+    const int64_t q0 = __ldg(a.qoff + b), qn = __ldg(a.qoff + b + 1) - q0;
+    if (qn < 1) continue;
+    if (q0 < 0 || q0 >= a.total_q) continue;  // inconsistent offsets: reported by the combine
+    f(b, s, e, q0);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// bf16 split-context pass on the tensor cores (mma.sync m16n8k16).
+// Per warp and 16-key slice of a tile:  S^T[16 keys x 8 heads] = K Q^T, then
+// O^T[128 x 8] += V^T P^T, with P^T obtained from the S^T accumulator by one
+// register transpose (movmatrix), so no shared-memory round trip for P.
+// Warp 4 is the producer: one lane issues TMA loads into an NST-deep ring.
+// ----------------------------------------------------------------------------
+template <int NST>
+__global__ void __launch_bounds__(32 * (kDecWarps + 1))
+    k_decode_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ DecodeArgs a) {
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full_bar[NST];
+  __shared__ __align__(8) uint64_t empty_bar[NST];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = blockIdx.x, g = blockIdx.y;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kDecWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kDecWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    const uint64_t pol = policy_evict_first();
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0;  // bit s: stage s has a fill in flight or unconsumed
+    uint32_t last_phase = 0;
+    bool ok = true;
+    for_each_piece(a, p, [&](int b, int64_t s, int64_t e, int64_t q0) {
+      for (int64_t k0 = s; k0 < e && ok; k0 += kDecTile) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1)) {
+          record_error(a.err, HS2_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full_bar[stage], kDecStageBytes);
+        uint8_t* sk = ring + stage * kDecStageBytes;
+        uint8_t* sv = sk + 2 * 8192;
+        const int key = static_cast<int>(k0);
+        tma_load_3d_hint(sk, &tmK, &full_bar[stage], 0, g, key, pol);
+        tma_load_3d_hint(sk + 8192, &tmK, &full_bar[stage], 64, g, key, pol);
+        tma_load_3d_hint(sv, &tmV, &full_bar[stage], 0, g, key, pol);
+        tma_load_3d_hint(sv + 8192, &tmV, &full_bar[stage], 64, g, key, pol);
+        issued |= 1u << stage;
+        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == NST) { stage = 0; phase ^= 1; }
+      }
+    });
+    // drain: every fill this thread issued has landed before the CTA can exit
+    for (int s = 0; s < NST; ++s)
+      if ((issued >> s) & 1u)
+        if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) record_error(a.err, HS2_ERR_TIMEOUT);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const bf16* Q = static_cast<const bf16*>(a.Q);
+  const int r = lane >> 2, qd = lane & 3;
+  const float NEG = -INFINITY;
+  int stage = 0;
+  uint32_t phase = 0;
+  bool ok = true;
+
+  for_each_piece(a, p, [&](int b, int64_t s, int64_t e, int64_t q0) {
+    // query fragments: B operand of S^T = K Q^T, head n = r of the group
+    uint32_t qf[8][2];
+    const bf16* qrow = Q + ((q0 * a.Hq) + (int64_t)g * a.G + r) * kD;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      if (r < a.G) {
+        qf[kk][0] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * qd);
+        qf[kk][1] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * qd);
+      } else {
+        qf[kk][0] = qf[kk][1] = 0u;
+      }
+    }
+    float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
+    float o[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+
+    const int h0 = 2 * qd, h1 = 2 * qd + 1;  // this thread's two heads
+    float* lg = a.logits + (int64_t)g * a.G;
+
+    for (int64_t k0 = s; k0 < e; k0 += kDecTile) {
+      if (ok && !mbar_wait(&full_bar[stage], phase)) {
+        record_error(a.err, HS2_ERR_TIMEOUT);
+        ok = false;
+      }
+      if (ok) {
+        const uint8_t* sk = ring + stage * kDecStageBytes;
+        const uint8_t* sv = sk + 2 * 8192;
+        const uint32_t skb = smem_u32(sk), svb = smem_u32(sv);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const int row = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const int chunk = (kk & 3) * 2 + (lane >> 4);
+            const uint32_t addr = skb + (kk >> 2) * 8192 + row * 128 + ((chunk ^ (row & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(a0, a1, a2, a3, addr);
+            mma_bf16(c, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+          }
+        }
+        const int64_t klo = k0 + warp * 16 + r, khi = klo + 8;
+        const bool vlo = klo < e, vhi = khi < e;
+        const float x0 = vlo ? c[0] * a.scale : NEG, x1 = vlo ? c[1] * a.scale : NEG;
+        const float x2 = vhi ? c[2] * a.scale : NEG, x3 = vhi ? c[3] * a.scale : NEG;
+        // logits of the real heads
+        if (h1 < a.G && (a.G & 1) == 0) {  // even G: the pair is 8-byte aligned
+          if (vlo) *reinterpret_cast<float2*>(lg + klo * a.Hq + h0) = make_float2(x0, x1);
+          if (vhi) *reinterpret_cast<float2*>(lg + khi * a.Hq + h0) = make_float2(x2, x3);
+        } else {
+          if (h0 < a.G) {
+            if (vlo) lg[klo * a.Hq + h0] = x0;
+            if (vhi) lg[khi * a.Hq + h0] = x2;
+          }
+          if (h1 < a.G) {
+            if (vlo) lg[klo * a.Hq + h1] = x1;
+            if (vhi) lg[khi * a.Hq + h1] = x3;
+          }
+        }
+        // online softmax over the 16 keys of this warp, per head (column)
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float al0 = (mn0 == NEG) ? 1.f : exp_shift(m0, mn0);
+        const float al1 = (mn1 == NEG) ? 1.f : exp_shift(m1, mn1);
+        const float p0 = exp_shift(x0, mn0), p1 = exp_shift(x1, mn1);
+        const float p2 = exp_shift(x2, mn0), p3 = exp_shift(x3, mn1);
+        l0 = l0 * al0 + (p0 + p2);
+        l1 = l1 * al1 + (p1 + p3);
+        m0 = mn0;
+        m1 = mn1;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          o[i][0] *= al0; o[i][1] *= al1; o[i][2] *= al0; o[i][3] *= al1;
+        }
+        const uint32_t b0 = movmatrix_t(pack_bf16(p0, p1));
+        const uint32_t b1 = movmatrix_t(pack_bf16(p2, p3));
+        {
+          const int row = warp * 16 + ((lane >> 4) & 1) * 8 + (lane & 7);
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            const int chunk = (mt & 3) * 2 + ((lane >> 3) & 1);
+            const uint32_t addr = svb + (mt >> 2) * 8192 + row * 128 + ((chunk ^ (row & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(a0, a1, a2, a3, addr);
+            mma_bf16(o[mt], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[stage]);
+      if (++stage == NST) { stage = 0; phase ^= 1; }
+    }
+    // per-warp partial of this piece
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    const int64_t slot = (int64_t)p + b;
+    const int64_t base = ((slot * a.Hkv + g) * kDecWarps + warp) * a.G;
+    if (r == 0) {
+      if (h0 < a.G) { a.pm[base + h0] = m0; a.pl[base + h0] = l0; }
+      if (h1 < a.G) { a.pm[base + h1] = m1; a.pl[base + h1] = l1; }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      const int d = mt * 16 + r;
+      if (h0 < a.G) {
+        a.po[(base + h0) * kD + d] = o[mt][0];
+        a.po[(base + h0) * kD + d + 8] = o[mt][2];
+      }
+      if (h1 < a.G) {
+        a.po[(base + h1) * kD + d] = o[mt][1];
+        a.po[(base + h1) * kD + d + 8] = o[mt][3];
+      }
+    }
+  });
+}
+
+// ----------------------------------------------------------------------------
+// float32 split-context pass on the CUDA cores (exact fp32 products and sums).
+// Each warp takes every 4th key of the CTA's pieces; lane i holds dims
+// 4i..4i+3.  GP >= G is the compile-time head bound.
+// ----------------------------------------------------------------------------
+template <int GP>
+__global__ void __launch_bounds__(32 * kDecWarps) k_decode_f32(const __grid_constant__ DecodeArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = blockIdx.x, g = blockIdx.y;
+  const float* Q = static_cast<const float*>(a.Q);
+  const float* K = static_cast<const float*>(a.K);
+  const float* V = static_cast<const float*>(a.V);
+  for_each_piece(a, p, [&](int b, int64_t s, int64_t e, int64_t q0) {
+    float4 q[GP];
+    float m[GP], l[GP];
+    float4 o[GP];
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+      q[h] = (h < a.G) ? *reinterpret_cast<const float4*>(Q + ((q0 * a.Hq) + (int64_t)g * a.G + h) * kD + lane * 4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+      o[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int64_t j = s + warp; j < e; j += kDecWarps) {
+      const float4 kv = *reinterpret_cast<const float4*>(K + (j * a.Hkv + g) * kD + lane * 4);
+      const float4 vv = *reinterpret_cast<const float4*>(V + (j * a.Hkv + g) * kD + lane * 4);
+#pragma unroll
+      for (int h = 0; h < GP; ++h) {
+        if (h >= a.G) break;
+        float dot = q[h].x * kv.x;
+        dot = fmaf(q[h].y, kv.y, dot);
+        dot = fmaf(q[h].z, kv.z, dot);
+        dot = fmaf(q[h].w, kv.w, dot);
+        const float x = warp_sum(dot) * a.scale;
+        if (lane == 0) a.logits[j * a.Hq + (int64_t)g * a.G + h] = x;
+        const float mn = fmaxf(m[h], x);
+        const float al = exp_shift(m[h], mn);
+        const float pr = expf(x - mn);
+        l[h] = l[h] * al + pr;
+        o[h].x = fmaf(pr, vv.x, o[h].x * al);
+        o[h].y = fmaf(pr, vv.y, o[h].y * al);
+        o[h].z = fmaf(pr, vv.z, o[h].z * al);
+        o[h].w = fmaf(pr, vv.w, o[h].w * al);
+        m[h] = mn;
+      }
+    }
+    const int64_t slot = (int64_t)p + b;
+    const int64_t base = ((slot * a.Hkv + g) * kDecWarps + warp) * a.G;
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+      if (h >= a.G) break;
+      if (lane == 0) { a.pm[base + h] = m[h]; a.pl[base + h] = l[h]; }
+      *reinterpret_cast<float4*>(a.po + (base + h) * kD + lane * 4) = o[h];
+    }
+  });
+}
+
+// ----------------------------------------------------------------------------
+// Combine: O and (m_h, l_h) of each (sequence, head) from the per-warp partials
+// of every CTA whose key range meets the sequence.  Grid (B, Hkv), D threads.
+// ----------------------------------------------------------------------------
+template <typename OT>
+__global__ void __launch_bounds__(kD) k_decode_combine(const __grid_constant__ DecodeArgs a, OT* O,
+                                                       float* ml) {
+  const int b = blockIdx.x, g = blockIdx.y, d = threadIdx.x;
+  if (b == 0 && g == 0 && d == 0) {
+    if (__ldg(a.kvoff + a.B) != a.total_kv || __ldg(a.qoff + a.B) != a.total_q)
+      record_error(a.err, HS2_ERR_DEVICE_INPUT);
+  }
+  const int64_t q0 = __ldg(a.qoff + b);
+  const int64_t qn = __ldg(a.qoff + b + 1) - q0;
+  if (qn < 1) return;
+  if (qn > 1 || q0 < 0 || q0 >= a.total_q) {
+    if (d == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+    return;
+  }
+  const int64_t W = a.total_kv;
+  const int64_t kb = __ldg(a.kvoff + b), ke = __ldg(a.kvoff + b + 1);
+  int pf = 0, pe = -1;
+  if (ke > kb) {
+    pf = split_owner(W, a.P, kb);
+    pe = split_owner(W, a.P, ke - 1);
+  }
+  for (int hl = 0; hl < a.G; ++hl) {
+    float M = -INFINITY;
+    for (int p = pf; p <= pe; ++p) {
+      if (split_lo(W, a.P, p) == split_lo(W, a.P, p + 1)) continue;
+      const int64_t base = (((int64_t)(p + b) * a.Hkv + g) * kDecWarps) * a.G + hl;
+      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, a.pm[base + w * a.G]);
+    }
+    float L = 0.f, acc = 0.f;
+    for (int p = pf; p <= pe; ++p) {
+      if (split_lo(W, a.P, p) == split_lo(W, a.P, p + 1)) continue;
+      const int64_t base = (((int64_t)(p + b) * a.Hkv + g) * kDecWarps) * a.G + hl;
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float wt = exp_shift(a.pm[base + w * a.G], M);
+        L = fmaf(a.pl[base + w * a.G], wt, L);
+        acc = fmaf(a.po[(base + w * a.G) * kD + d], wt, acc);
+      }
+    }
+    const int64_t row = q0 * a.Hq + (int64_t)g * a.G + hl;
+    O[row * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
+    if (d == 0) {
+      ml[row * 2] = M;
+      ml[row * 2 + 1] = L;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Scores: s_g[j] = sum_{h in group g} exp(x_hj - m_h) / l_h, written to row
+// (query, g) at column j (position within the sequence).  64 keys per block,
+// threads (key, group) so that each warp writes 32 consecutive scores.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_finalize_scores(const __grid_constant__ DecodeArgs a,
+                                                         const float* ml, float* scores,
+                                                         int64_t stride) {
+  const int kl = threadIdx.x & 63;
+  const int64_t key = (int64_t)blockIdx.x * 64 + kl;
+  if (key >= a.total_kv) return;
+  const int b = last_le(a.kvoff, a.B, key);
+  const int64_t q0 = __ldg(a.qoff + b);
+  if (__ldg(a.qoff + b + 1) - q0 < 1) return;
+  const int64_t j = key - __ldg(a.kvoff + b);
+  if (q0 < 0 || q0 >= a.total_q || j < 0 || j >= stride) {
+    record_error(a.err, HS2_ERR_DEVICE_INPUT);
+    return;
+  }
+  for (int g = threadIdx.x >> 6; g < a.Hkv; g += 4) {
+    const float* x = a.logits + key * a.Hq + (int64_t)g * a.G;
+    const float* st = ml + (q0 * a.Hq + (int64_t)g * a.G) * 2;
+    float s = 0.f;
+    for (int h = 0; h < a.G; ++h) s += expf(x[h] - st[2 * h]) / st[2 * h + 1];
+    scores[(q0 * a.Hkv + g) * stride + j] = s;
+  }
+}
+
+}  // namespace hs2

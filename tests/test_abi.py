@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every function include/hs2.h declares, and
+rejects bad arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_full_b200 import hs2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hs2.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hs2_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_full_b200 import build
+    build.build()
+    return hs2.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "hs2_full_attn_scores" in names and "hs2_topk_select" in names
+    assert "hs2_sparse_attn" in names and "hs2_block_select" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(hs2.EXPORTED) == names
+
+
+def test_status_strings_and_version(lib):
+    assert hs2.status_string(0) == "ok"
+    for code in range(-6, 0):
+        assert hs2.status_string(code) not in ("ok", "unknown status")
+    assert hs2.status_string(-99) == "unknown status"
+    assert hs2.hs2_version() >= 1
+
+
+def _problem(**kw):
+    d = dict(B=1, Hq=8, Hkv=2, D=128, dtype=hs2.HS2_BF16, q_offsets=0x1000, kv_offsets=0x2000,
+             total_q=1, total_kv=100, max_q_len=1, max_kv_len=100, scale=0.0884)
+    d.update(kw)
+    return hs2.make_problem(**d)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=7), hs2.HS2_ERR_INVALID_ARG),          # Hq % Hkv != 0
+    (dict(B=0), hs2.HS2_ERR_INVALID_ARG),
+    (dict(dtype=5), hs2.HS2_ERR_INVALID_ARG),
+    (dict(q_offsets=None), hs2.HS2_ERR_INVALID_ARG),
+    (dict(total_kv=1000), hs2.HS2_ERR_INVALID_ARG),   # more keys than B * max_kv_len
+    (dict(max_q_len=200), hs2.HS2_ERR_INVALID_ARG),   # queries longer than the cache
+    (dict(scale=float("nan")), hs2.HS2_ERR_INVALID_ARG),
+    (dict(D=64), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(Hq=32, Hkv=2), hs2.HS2_ERR_UNSUPPORTED),    # bf16 group of 16 heads
+])
+def test_problem_validation(lib, kw, code):
+    p = _problem(**kw)
+    n = ctypes.c_size_t(0)
+    assert lib.hs2_topk_workspace_size(ctypes.byref(p), 1024, 128, ctypes.byref(n)) == code
+    assert lib.hs2_full_attn_workspace_size(ctypes.byref(p), ctypes.byref(n)) == code
+    rc = lib.hs2_topk_select(ctypes.byref(p), 0x3000, 128, 1024, 128, 0x4000, 0x5000, None, 0, None)
+    assert rc == code
+
+
+def test_null_problem_and_bad_call_arguments(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.hs2_topk_workspace_size(None, 1024, 128, ctypes.byref(n)) == hs2.HS2_ERR_INVALID_ARG
+    p = _problem()
+    assert lib.hs2_topk_workspace_size(ctypes.byref(p), 0, 128, ctypes.byref(n)) == hs2.HS2_ERR_INVALID_ARG
+    # score stride shorter than the longest sequence
+    assert lib.hs2_topk_select(ctypes.byref(p), 0x3000, 50, 1024, 128, 0x4000, 0x5000, None, 0,
+                               None) == hs2.HS2_ERR_INVALID_ARG
+    # misaligned scores pointer
+    assert lib.hs2_topk_select(ctypes.byref(p), 0x3004, 128, 1024, 128, 0x4000, 0x5000, None, 0,
+                               None) == hs2.HS2_ERR_INVALID_ARG
+    # null outputs
+    assert lib.hs2_full_attn_scores(ctypes.byref(p), 0x1000, 0x1000, 0x1000, None, 0x1000, 128,
+                                    None, 0, None) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_topk_workspace_size_formula(lib):
+    # histogram (2048 x 4 B) + ticket + prefix + krem + per-slice counts, each 256-B rounded
+    p = _problem(total_q=3, B=3, max_kv_len=10000, total_kv=20000)
+    n = ctypes.c_size_t(0)
+    assert lib.hs2_topk_workspace_size(ctypes.byref(p), 1024, 128, ctypes.byref(n)) == 0
+    rows = 3 * 2
+    rnd = lambda b: (b + 255) // 256 * 256
+    slices = (10000 + 4095) // 4096
+    want = rnd(rows * 2048 * 4) + 3 * rnd(rows * 4) + rnd(rows * slices * 2 * 4)
+    assert n.value == want

@@ -1,0 +1,201 @@
+"""CUDA path vs the CPU oracle on the same seeded inputs (small and mid sizes:
+several tiles, ragged tails, edge lengths, ties, grouped-query variants)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from long_context_full_b200 import hs2
+from tests.gpu_util import (GpuRun, OracleRows, check_O, check_index_sets, check_scores,
+                            gpu_select_on, to_device, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def full_check(w, select="token", rows=None, layers=True):
+    """Runs the CUDA path and checks O, scores, selection and sparse layers for
+    the listed query rows (all by default).  Returns a summary dict."""
+    run = GpuRun(w, select)
+    out = run.run()
+    ora = OracleRows(w)
+    O = out.O
+    S = out.scores.cpu().numpy()
+    idx = out.idx.cpu().numpy()
+    cnt = out.count.cpu().numpy()
+    OL = [to_f64(x) for x in out.O_layers] if layers else None
+    Og = to_f64(O)
+    rows = range(w.q.shape[0]) if rows is None else rows
+    summ = dict(o_err=0.0, score_rel=0.0, flips=0, sparse_err=0.0)
+    for r in rows:
+        Oref, sref, t = ora.full(r)
+        summ["o_err"] = max(summ["o_err"], check_O(Og[r], Oref, w.dtype, f"O row {r}"))
+        for g in range(w.Hkv):
+            R = r * w.Hkv + g
+            summ["score_rel"] = max(summ["score_rel"],
+                                    check_scores(S[R, :t + 1], sref[g], f"scores row {r} g {g}"))
+            # selection on the oracle's own scores is bit-exact
+            if select == "token":
+                oi, oc = oracle.topk_select(sref[g], t, w.topk, w.window)
+            else:
+                oi, oc = oracle.block_select(sref[g], t, w.n_blocks, w.block, w.window)
+            if select == "token":
+                summ["flips"] += check_index_sets(idx[R], int(cnt[R]), oi, oc, sref[g], t, w.topk,
+                                                  w.window, f"indices row {r} g {g}")
+            else:
+                assert int(cnt[R]) == oc
+        if layers:
+            sets = [idx[r * w.Hkv + g, :cnt[r * w.Hkv + g]] for g in range(w.Hkv)]
+            for l in range(w.n_layers):
+                ref = ora.sparse(r, l, sets)
+                summ["sparse_err"] = max(summ["sparse_err"],
+                                         check_O(OL[l][r], ref, w.dtype, f"layer {l} row {r}"))
+    return summ, out
+
+
+def test_tiny_f32_workload():
+    """Batch 1, one decode query over 4096 keys, Hq=4 / Hkv=1, fp32, 3 reuse layers."""
+    w = synth.tiny()
+    summ, out = full_check(w)
+    assert summ["flips"] == 0
+    assert int(out.count[0]) == 1152
+
+
+def test_sparse_equals_full_when_budget_covers_context():
+    """t + 1 <= 1024 + 128: the index set is the whole context, so a sparse layer
+    given the full-attention layer's query reproduces the full output."""
+    for dtype in ("f32", "bf16"):
+        w = synth.make_workload("short", 11, dtype, 8, 2, 128, [1152, 700, 1], [1, 1, 1], 1)
+        w.q_layers[0][:] = w.q  # same queries as the full-attention layer
+        run = GpuRun(w)
+        out = run.run()
+        cnt = out.count.cpu().numpy()
+        assert list(cnt) == [1152, 1152, 700, 700, 1, 1]
+        a, b = to_f64(out.O), to_f64(out.O_layers[0])
+        tol = 2e-2 if dtype == "bf16" else 1e-5
+        assert np.abs(a - b).max() <= tol * (1 if dtype == "bf16" else np.abs(a).max())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_ragged_decode_edge_lengths(dtype):
+    lens = [1, 2, 127, 128, 129, 1151, 1152, 1153, 1280, 4096, 9000]
+    w = synth.make_workload("edges", 21, dtype, 16, 2, 128, lens, [1] * len(lens), 2)
+    summ, out = full_check(w)
+    cnt = out.count.cpu().numpy().reshape(-1, 2)[:, 0]
+    assert list(cnt) == [min(n, 1152) for n in lens]
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv", [("bf16", 4, 4), ("bf16", 8, 4), ("bf16", 8, 2),
+                                          ("bf16", 32, 4), ("f32", 4, 1), ("f32", 16, 2),
+                                          ("f32", 16, 1), ("f32", 6, 2)])
+def test_gqa_variants(dtype, Hq, Hkv):
+    w = synth.make_workload("gqa", 31, dtype, Hq, Hkv, 128, [3000, 1500], [1, 1], 1)
+    full_check(w)
+
+
+def test_decode_many_tiles_bf16():
+    """Two sequences long enough for every CTA of the split to see several
+    tiles and a ragged tail, batch boundary inside a CTA range."""
+    w = synth.make_workload("mid", 41, "bf16", 32, 4, 128, [70001, 33333], [1, 1], 2)
+    summ, _ = full_check(w)
+    assert summ["score_rel"] < 2e-5
+
+
+def _select_rows():
+    rng = np.random.default_rng(5)
+    n = 20000
+    rows = [
+        np.ones(n, np.float32),                                      # all equal
+        np.arange(n, dtype=np.float32),                              # strictly increasing
+        rng.integers(0, 3, n).astype(np.float32),                    # heavy ties at threshold
+        rng.random(n).astype(np.float32),                            # distinct
+        np.where(rng.random(n) < 0.5, np.float32(0.0), np.float32(-0.0)),  # +0 / -0
+        (rng.random(n) * 2 - 1).astype(np.float32),                 # negatives
+    ]
+    x = rng.random(n).astype(np.float32)
+    x[rng.choice(n, 3000, replace=False)] = np.float32(0.75)         # a big block of equal values
+    rows.append(x)
+    return np.stack(rows)
+
+
+def test_select_bit_exact_on_fixed_scores():
+    S = _select_rows()
+    ts = [19999, 19999, 15000, 19999, 19999, 12345, 19999]
+    idx, cnt = gpu_select_on(S, ts)
+    for r, t in enumerate(ts):
+        oi, oc = oracle.topk_select(S[r], t)
+        assert int(cnt[r]) == oc
+        assert np.array_equal(idx[r], oi), f"row {r}"
+
+
+@pytest.mark.parametrize("t", [0, 1, 126, 127, 128, 129, 1151, 1152, 1153, 4223, 4224, 4225, 8319, 70000])
+def test_select_edge_positions(t):
+    rng = np.random.default_rng(t)
+    s = rng.integers(0, 50, t + 1).astype(np.float32)
+    idx, cnt = gpu_select_on(s[None, :], [t])
+    oi, oc = oracle.topk_select(s, t)
+    assert int(cnt[0]) == oc and np.array_equal(idx[0], oi)
+
+
+def test_block_select_bit_exact():
+    S = _select_rows()
+    ts = [19999, 19999, 15000, 19999, 19999, 12345, 19999]
+    idx, cnt = gpu_select_on(S, ts, block_mode=True)
+    for r, t in enumerate(ts):
+        oi, oc = oracle.block_select(S[r], t)
+        assert int(cnt[r]) == oc
+        assert np.array_equal(idx[r], oi), f"row {r}"
+    for t in (0, 5, 127, 128, 191, 192, 1151, 1152, 1153, 1200, 5000):
+        s = np.random.default_rng(t).random(t + 1).astype(np.float32)
+        i, c = gpu_select_on(s[None, :], [t], block_mode=True)
+        oi, oc = oracle.block_select(s, t)
+        assert int(c[0]) == oc and np.array_equal(i[0], oi), t
+
+
+def test_block_select_path_end_to_end():
+    w = synth.make_workload("blk", 51, "bf16", 16, 2, 128, [5000, 2000, 300], [1, 1, 1], 1)
+    full_check(w, select="block")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_chunk_causal(dtype):
+    """Several new query tokens per sequence on top of a cached context."""
+    w = synth.make_workload("chunk", 61, dtype, 16, 2, 128, [3000, 1500, 300], [200, 37, 300], 1)
+    full_check(w)
+
+
+def test_chunk_gqa_bf16():
+    for Hq, Hkv in ((4, 4), (8, 2), (32, 4)):
+        w = synth.make_workload("chunkg", 62, "bf16", Hq, Hkv, 128, [2500], [150], 1)
+        full_check(w)
+
+
+def test_repeatable():
+    w = synth.make_workload("rep", 71, "bf16", 32, 4, 128, [50000, 20000], [1, 1], 1)
+    run = GpuRun(w)
+    a = run.run()
+    i1, s1, o1 = a.idx.clone(), a.scores.clone(), a.O_layers[0].clone()
+    b = run.run()
+    assert torch.equal(i1, b.idx) and torch.equal(s1, b.scores) and torch.equal(o1, b.O_layers[0])
+
+
+def test_device_input_errors_are_reported():
+    w = synth.make_workload("err", 81, "bf16", 8, 1, 128, [500], [1], 1)
+    run = GpuRun(w)
+    run.run()
+    bad = run.step.idx.clone()
+    bad[0, 3] = 600  # beyond the query position
+    hs2.hs2_sparse_attn(run.step.problem, run.QL[0], run.K, run.V, bad, run.step.count,
+                        run.step.idx_stride, run.step.O_layers[0], run.step.workspace)
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_ERR_DEVICE_INPUT
+    assert torch.isfinite(run.step.O_layers[0].float()).all()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK  # cleared
+
+
+def test_host_checks_launch_nothing():
+    w = synth.make_workload("chk", 91, "bf16", 8, 1, 128, [500], [1], 1)
+    run = GpuRun(w)
+    with pytest.raises(hs2.HS2Error) as e:
+        hs2.hs2_topk_select(run.step.problem, run.step.scores, run.step.stride, 1024, 128,
+                            run.step.idx, run.step.count, None)
+    assert e.value.status == hs2.HS2_ERR_WORKSPACE
