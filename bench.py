@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Throughput of one HySparse2 hybrid-block decode step on B200.
+
+A step is one pass of the whole path over one batch: the full-attention
+layer over the shared KV cache with per-key selection scores, token-level
+top-1024 + 128-window selection, and 4 sparse-attention layers that reuse the
+cache and the indices.  Workload per GPU (weak scaling, independent sequences,
+no collective on the data path): 8 decode sequences x 131072 cached tokens,
+32 query / 4 KV heads, head dim 128, bf16, synthetic N(0,1) inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torch.distributed.run (one process per GPU, NCCL only
+for the barrier and the max-over-ranks timing).  Rank 0 prints one JSON line.
+``--impl reference`` times the CPU oracle (float64, the host cores) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "query-tok/s & KV-scan HBM GB/s (vs ~8 TB/s), select+sparse attn, 128K–1M ctx"
+UNIT = "query-tok/s"
+BATCH, CONTEXT, HQ, HKV, D, LAYERS, TOPK, WINDOW = 8, 131072, 32, 4, 128, 4, 1024, 128
+WORKLOAD = "decode_b8_128k_bf16"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=BATCH,
+                    help="sequences per GPU (smaller only for profiling captures)")
+    ap.add_argument("--context", type=int, default=CONTEXT,
+                    help="cached tokens per sequence (smaller only for profiling captures)")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+# ---------------------------------------------------------------------------
+# workload accounting
+# ---------------------------------------------------------------------------
+def algorithmic_bytes(batch=BATCH, context=CONTEXT, count=TOPK + WINDOW):
+    """Bytes the step must move at least once (bf16 cache, fp32 scores).
+
+    full attention: K and V read once, Q read, O written, scores written;
+    selection: scores read once; each sparse layer: the selected K/V rows
+    gathered once, its Q read and O written."""
+    kv = 2 * batch * context * HKV * D * 2
+    q = batch * HQ * D * 2
+    scores = batch * HKV * context * 4
+    gather = batch * HKV * count * D * 2 * 2
+    full = kv + 2 * q + scores
+    select = scores + batch * HKV * (count + 1) * 4
+    sparse = gather + 2 * q
+    return dict(full=full, select=select, sparse_layer=sparse,
+                step=full + select + LAYERS * sparse, kv=kv)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(kernel_src_hash: str):
+    """DRAM bytes per launch of the full-attention call from the committed ncu
+    summary, or None if it was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "full_attn_decode_b8_128k.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_call:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_sources_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != kernel_src_hash:
+        return None
+    return float(m.group(1))
+
+
+def kernel_sources_hash() -> str:
+    csrc = os.path.join(ROOT, "long_context_full_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML sampler thread)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period: float = 0.02):
+        self.samples, self.reasons = [], 0
+        self.ok = False
+        self.max_mhz = None
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if not self.ok:
+            return None
+        self._stop.set()
+        self._t.join()
+        self._sample()
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (the baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_unit(w, r: int, g: int, n_keys: int | None = None):
+    """The oracle's full step for one (query row, KV group): full attention of
+    the group's heads over the first n_keys cached tokens (all by default),
+    scores, top-k select, and every sparse layer."""
+    import oracle
+    import synth
+    b = int(w.query_seq()[r])
+    ko = w.kv_offsets
+    n = int(w.kv_lens[b]) if n_keys is None else n_keys
+    G = w.Hq // w.Hkv
+    ks = synth.stored_to_f64(w.k[ko[b]:ko[b] + n, g:g + 1], w.dtype)
+    vs = synth.stored_to_f64(w.v[ko[b]:ko[b] + n, g:g + 1], w.dtype)
+    q = synth.stored_to_f64(w.q[r, g * G:(g + 1) * G], w.dtype)
+    t = n - 1
+    O, m, l, P = oracle.full_attention_row(q, ks, vs, t, w.scale)
+    s = oracle.selection_scores(P, 1)
+    idx, c = oracle.topk_select(s[0], t, w.topk, w.window)
+    for layer in range(w.n_layers):
+        ql = synth.stored_to_f64(w.q_layers[layer][r, g * G:(g + 1) * G], w.dtype)
+        oracle.sparse_attention_row(ql, ks, vs, [idx[:c]], w.scale)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(w, budget_s: float = 12.0):
+    """Oracle throughput in query-tok/s on whole (query, KV group) units until
+    ``budget_s`` of CPU time has been spent (at least one unit)."""
+    units, t0 = 0, time.perf_counter()
+    for r in range(w.q.shape[0]):
+        for g in range(w.Hkv):
+            oracle_unit(w, r, g)
+            units += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": (units / w.Hkv) / dt, "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{units} (query, KV-group) units of {w.q.shape[0] * w.Hkv}: full attention "
+                      f"of the group's {w.Hq // w.Hkv} heads over {int(w.kv_lens[0])} keys, scores, top-k "
+                      f"select, {w.n_layers} sparse layers; float64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle as it stands, on a bounded sample of
+    this workload; rank 0 only."""
+    if rank != 0:
+        return
+    import synth
+    w = synth.decode_128k(batch=1)
+    # sample size per step: one (query, KV group) unit over the first n_keys
+    # cached tokens, shrunk so that all steps fit in about two minutes
+    t0 = time.perf_counter()
+    oracle_unit(w, 0, 0)
+    unit_s = time.perf_counter() - t0
+    steps = args.steps + args.warmup
+    n_keys = CONTEXT
+    if steps * unit_s > 120.0:
+        n_keys = max(4096, int(CONTEXT * 120.0 / (steps * unit_s)))
+    for _ in range(args.warmup):
+        oracle_unit(w, 0, 0, n_keys)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_unit(w, 0, i % HKV, n_keys)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    # throughput of the sample scaled to whole queries over the full context
+    value = (1.0 / HKV) * (n_keys / CONTEXT) / dt
+    sample = (f"one (query, KV group) unit per step: full attention of 8 heads over the first "
+              f"{n_keys} of {CONTEXT} keys, scores, top-k select, {LAYERS} sparse layers; "
+              f"value scaled by (1/{HKV}) x ({n_keys}/{CONTEXT}) per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "batch_per_gpu": BATCH, "context": CONTEXT,
+                       "Hq": HQ, "Hkv": HKV, "D": D, "k": TOPK, "window": WINDOW,
+                       "reuse_layers": LAYERS},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import synth
+    from long_context_full_b200 import hs2
+    from long_context_full_b200.block import HybridBlockStep
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    hs2.load()
+
+    batch, context = args.batch, args.context
+    w = synth.decode_128k(batch=batch, first_seq=rank * batch, context=context)
+    workload = WORKLOAD if (batch, context) == (BATCH, CONTEXT) else \
+        f"decode_b{batch}_{context}_bf16 (profiling case)"
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    Q, K, V = dev(w.q), dev(w.k), dev(w.v)
+    QL = [dev(x) for x in w.q_layers]
+    step = HybridBlockStep(HQ, HKV, D, torch.bfloat16, w.q_lens, w.kv_lens, LAYERS, k=TOPK,
+                           window=WINDOW)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- warm-up
+    for _ in range(max(3, args.warmup)):
+        step.run(Q, K, V, QL)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+
+    # ---- device-timed region: exactly K steps, events per phase
+    Kst = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(Kst)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(stream)
+    for i in range(Kst):
+        e = ev[i]
+        e[0].record(stream)
+        step.full_attention(Q, K, V)
+        e[1].record(stream)
+        step.select_tokens()
+        e[2].record(stream)
+        for layer in range(LAYERS):
+            step.sparse_layer(layer, QL[layer], K, V)
+        e[3].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    ph = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+                   for e in ev])
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    elapsed_ms = max_over_ranks(elapsed_ms)
+    ms_step = elapsed_ms / Kst
+    value = batch * world * Kst / (elapsed_ms / 1e3)
+
+    ab = algorithmic_bytes(batch, context)
+    t_full = float(ph[:, 0].mean())
+    t_sel = float(ph[:, 1].mean())
+    t_sp = float(ph[:, 2].mean())
+    hbm, hbm_kind = peaks()
+    achieved = ab["full"] / (t_full * 1e-3) / 1e9
+    traffic = profiled_traffic(kernel_sources_hash())
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hQ, hK, hV = pin(w.q), pin(w.k), pin(w.v)
+    hQL = [pin(x) for x in w.q_layers]
+    outs = [step.O] + step.O_layers + [step.idx, step.count]
+    hout = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    h2d = sum(t.numel() * t.element_size() for t in [hQ, hK, hV] + hQL)
+    d2h = sum(t.numel() * t.element_size() for t in hout)
+
+    def e2e_step():
+        for d_, h_ in zip([Q, K, V] + QL, [hQ, hK, hV] + hQL):
+            d_.copy_(h_, non_blocking=True)
+        step.run(Q, K, V, QL)
+        for h_, d_ in zip(hout, outs):
+            h_.copy_(d_, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    E = max(1, min(args.e2e_steps, Kst))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = batch * world * E / (e2e_ms / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": Kst,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) Q/K/V, Philox streams)",
+            "config": {"workload": workload, "batch_per_gpu": batch, "context": context,
+                       "Hq": HQ, "Hkv": HKV, "D": D, "k": TOPK, "window": WINDOW,
+                       "reuse_layers": LAYERS,
+                       "l2": f"inputs larger than L2: {ab['kv'] / 2**30:.2f} GiB of K/V streamed per step",
+                       "parallelism": f"dp{world} (independent sequences per GPU)"},
+            "kv_scan_gbs": ab["kv"] / (t_full * 1e-3) / 1e9,
+            "step_gbs": ab["step"] / (ms_step * 1e-3) / 1e9,
+            "phase_ms": {"full_attn_scores": t_full, "topk_select": t_sel,
+                         "sparse_attn_x4": t_sp},
+            "roofline": {"kernel": "hs2_full_attn_scores (decode pass + combine + score finalize)",
+                         "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "peak_kind": hbm_kind,
+                         "traffic": traffic, "algorithmic_bytes": ab["full"],
+                         "frac_of_8TBps": achieved / 8000.0},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": E},
+            "gpu_launches": Kst * step.launches_per_step(),
+            "clocks": clk,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

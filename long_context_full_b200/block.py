@@ -107,7 +107,7 @@ class HybridBlockStep:
         return StepOutputs(self.O, self.scores, self.idx, self.count, self.O_layers)
 
     def launches_per_step(self) -> int:
-        """Kernels one ``run`` launches (memsets excluded)."""
+        """Kernels one ``run`` launches."""
         full = 3 if self.max_q <= 1 else 2
-        sel = 5 if self.select == "token" else 7
+        sel = 1 if self.select == "token" else 3
         return full + sel + self.n_layers

@@ -320,14 +320,18 @@ __global__ void __launch_bounds__(32 * kDecWarps) k_decode_f32(const __grid_cons
 }
 
 // ----------------------------------------------------------------------------
-// Combine: O and (m_h, l_h) of each (sequence, head) from the per-warp partials
-// of every CTA whose key range meets the sequence.  Grid (B, Hkv), D threads.
+// Combine: O and (m_h, 1/l_h) of each (sequence, head) from the per-warp partials
+// of every CTA whose key range meets the sequence.  Grid (B, Hkv, G), D
+// threads: thread i owns partial i for the max and the weights, then thread d
+// sums dimension d over all partials (independent, coalesced loads).
 // ----------------------------------------------------------------------------
+constexpr int kCombStage = 64;  // partial rows staged in shared memory per round
+
 template <typename OT>
 __global__ void __launch_bounds__(kD) k_decode_combine(const __grid_constant__ DecodeArgs a, OT* O,
                                                        float* ml) {
-  const int b = blockIdx.x, g = blockIdx.y, d = threadIdx.x;
-  if (b == 0 && g == 0 && d == 0) {
+  const int b = blockIdx.x, g = blockIdx.y, hl = blockIdx.z, d = threadIdx.x;
+  if (b == 0 && g == 0 && hl == 0 && d == 0) {
     if (__ldg(a.kvoff + a.B) != a.total_kv || __ldg(a.qoff + a.B) != a.total_q)
       record_error(a.err, HS2_ERR_DEVICE_INPUT);
   }
@@ -335,68 +339,175 @@ __global__ void __launch_bounds__(kD) k_decode_combine(const __grid_constant__ D
   const int64_t qn = __ldg(a.qoff + b + 1) - q0;
   if (qn < 1) return;
   if (qn > 1 || q0 < 0 || q0 >= a.total_q) {
-    if (d == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+    if (d == 0 && hl == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
     return;
   }
   const int64_t W = a.total_kv;
   const int64_t kb = __ldg(a.kvoff + b), ke = __ldg(a.kvoff + b + 1);
-  int pf = 0, pe = -1;
+  int pf = 0, np = 0;
   if (ke > kb) {
     pf = split_owner(W, a.P, kb);
-    pe = split_owner(W, a.P, ke - 1);
+    np = (split_owner(W, a.P, ke - 1) - pf + 1) * kDecWarps;
   }
-  for (int hl = 0; hl < a.G; ++hl) {
-    float M = -INFINITY;
-    for (int p = pf; p <= pe; ++p) {
-      if (split_lo(W, a.P, p) == split_lo(W, a.P, p + 1)) continue;
-      const int64_t base = (((int64_t)(p + b) * a.Hkv + g) * kDecWarps) * a.G + hl;
-      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, a.pm[base + w * a.G]);
+  __shared__ __align__(16) float so[kCombStage][kD];
+  __shared__ float sw[kCombStage], swl[kCombStage];
+  __shared__ float red[kD / 32];
+  // partial i = (CTA pf + i / warps, warp i % warps); CTAs with an empty range wrote nothing
+  auto pidx = [&](int i, bool* valid) -> int64_t {
+    const int p = pf + i / kDecWarps;
+    *valid = split_lo(W, a.P, p) < split_lo(W, a.P, p + 1);
+    return (((int64_t)(p + b) * a.Hkv + g) * kDecWarps + (i % kDecWarps)) * a.G + hl;
+  };
+  float M = -INFINITY;
+  for (int i = d; i < np; i += kD) {
+    bool v;
+    const int64_t pi = pidx(i, &v);
+    if (v) M = fmaxf(M, a.pm[pi]);
+  }
+  M = warp_max(M);
+  if ((d & 31) == 0) red[d >> 5] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float L = 0.f, acc = 0.f;
+  for (int c0 = 0; c0 < np; c0 += kCombStage) {
+    const int n = min(kCombStage, np - c0);
+    if (d < n) {
+      bool v;
+      const int64_t pi = pidx(c0 + d, &v);
+      const float w = v ? exp_shift(a.pm[pi], M) : 0.f;
+      sw[d] = w;
+      swl[d] = w != 0.f ? w * a.pl[pi] : 0.f;
     }
-    float L = 0.f, acc = 0.f;
-    for (int p = pf; p <= pe; ++p) {
-      if (split_lo(W, a.P, p) == split_lo(W, a.P, p + 1)) continue;
-      const int64_t base = (((int64_t)(p + b) * a.Hkv + g) * kDecWarps) * a.G + hl;
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float wt = exp_shift(a.pm[base + w * a.G], M);
-        L = fmaf(a.pl[base + w * a.G], wt, L);
-        acc = fmaf(a.po[(base + w * a.G) * kD + d], wt, acc);
-      }
+    // the n partial O rows, all copies in flight at once (zero rows skipped)
+    for (int e = d; e < n * (kD / 4); e += kD) {
+      const int i = e / (kD / 4), c = e % (kD / 4);
+      bool v;
+      const int64_t pi = pidx(c0 + i, &v);
+      cp_async16(&so[i][c * 4], a.po + pi * kD + c * 4, v ? 16 : 0);
     }
-    const int64_t row = q0 * a.Hq + (int64_t)g * a.G + hl;
-    O[row * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
-    if (d == 0) {
-      ml[row * 2] = M;
-      ml[row * 2 + 1] = L;
+    cp_async_wait_all();
+    __syncthreads();
+    for (int i = 0; i < n; ++i) {
+      acc = fmaf(so[i][d], sw[i], acc);
+      L += swl[i];
     }
+    __syncthreads();
+  }
+  const int64_t row = q0 * a.Hq + (int64_t)g * a.G + hl;
+  O[row * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
+  if (d == 0) {  // (m_h, 1 / l_h): the score finalize multiplies
+    ml[row * 2] = M;
+    ml[row * 2 + 1] = L > 0.f ? 1.f / L : 0.f;
   }
 }
 
 // ----------------------------------------------------------------------------
 // Scores: s_g[j] = sum_{h in group g} exp(x_hj - m_h) / l_h, written to row
-// (query, g) at column j (position within the sequence).  64 keys per block,
-// threads (key, group) so that each warp writes 32 consecutive scores.
+// (query, g) at column j.  Persistent grid: block i handles key tiles i,
+// i + gridDim.x, ... of kFinKeys keys each (tile = (sequence, key block)).  A
+// tile's logits [keys x Hq] are one contiguous span; they are copied into
+// shared memory with 16-byte cp.async (row pitch Hq + 4 floats, so the per-key
+// reads below are free of bank conflicts), double-buffered so that the copy of
+// the next tile overlaps the exponentials of this one.  Thread j scores key j
+// of the tile for every KV head; the writes are coalesced along j.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_finalize_scores(const __grid_constant__ DecodeArgs a,
-                                                         const float* ml, float* scores,
-                                                         int64_t stride) {
-  const int kl = threadIdx.x & 63;
-  const int64_t key = (int64_t)blockIdx.x * 64 + kl;
-  if (key >= a.total_kv) return;
-  const int b = last_le(a.kvoff, a.B, key);
-  const int64_t q0 = __ldg(a.qoff + b);
-  if (__ldg(a.qoff + b + 1) - q0 < 1) return;
-  const int64_t j = key - __ldg(a.kvoff + b);
-  if (q0 < 0 || q0 >= a.total_q || j < 0 || j >= stride) {
-    record_error(a.err, HS2_ERR_DEVICE_INPUT);
-    return;
+constexpr int kFinKeys = 128;
+
+// Tile -> (sequence, first key); tiles cover ceil(max_len / kFinKeys) blocks
+// of every sequence, empty ones are skipped.
+__device__ __forceinline__ bool fin_tile(const DecodeArgs& a, int64_t tile, int ntile_seq, int* b,
+                                         int64_t* q0, int64_t* kb, int64_t* j0, int* nk) {
+  *b = (int)(tile / ntile_seq);
+  *j0 = (tile % ntile_seq) * kFinKeys;
+  *q0 = __ldg(a.qoff + *b);
+  if (__ldg(a.qoff + *b + 1) - *q0 < 1) return false;
+  *kb = __ldg(a.kvoff + *b);
+  const int64_t N = __ldg(a.kvoff + *b + 1) - *kb;
+  if (*j0 >= N) return false;
+  *nk = (int)(N - *j0 < kFinKeys ? N - *j0 : kFinKeys);
+  return true;
+}
+
+__global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_constant__ DecodeArgs a,
+                                                              const float* ml, float* scores,
+                                                              int64_t stride, int ntile_seq) {
+  extern __shared__ __align__(16) float fsm[];  // 2 x [kFinKeys][Hq + 4] logits, [Hq][2] stats
+  const int Hq = a.Hq, pitch = Hq + 4;
+  const int64_t ntiles = (int64_t)a.B * ntile_seq;
+  float* buf[2] = {fsm, fsm + (size_t)kFinKeys * pitch};
+  float* fst = fsm + 2 * (size_t)kFinKeys * pitch;  // (m_h, 1 / l_h) of the tile's query
+  const bool vec = (Hq & 3) == 0;
+  const bool vec4 = vec && (a.G & 3) == 0;
+
+  // issue the copy of one tile into buffer k (all threads)
+  auto load_tile = [&](int64_t tile, int k) -> bool {
+    int b, nk;
+    int64_t q0, kb, j0;
+    if (!fin_tile(a, tile, ntile_seq, &b, &q0, &kb, &j0, &nk)) return false;
+    const float* src = a.logits + (kb + j0) * Hq;
+    float* dst = buf[k];
+    if (vec) {
+      const int per_key = Hq / 4;
+      for (int i = threadIdx.x; i < nk * per_key; i += kFinKeys) {
+        const int key = i / per_key, c = i % per_key;
+        cp_async16(dst + key * pitch + c * 4, src + (int64_t)key * Hq + c * 4, 16);
+      }
+    } else {
+      for (int i = threadIdx.x; i < nk * Hq; i += kFinKeys) dst[(i / Hq) * pitch + i % Hq] = __ldg(src + i);
+    }
+    return true;
+  };
+
+  int64_t tile = blockIdx.x;
+  int cur = 0;
+  bool have = tile < ntiles && load_tile(tile, 0);
+  cp_async_commit();
+  while (tile < ntiles) {
+    const int64_t next = tile + gridDim.x;
+    // next non-empty tile goes into the other buffer while this one is scored
+    int64_t nt = next;
+    bool nhave = false;
+    while (nt < ntiles && !(nhave = load_tile(nt, cur ^ 1))) nt += gridDim.x;
+    cp_async_commit();
+    if (have) {
+      int b, nk;
+      int64_t q0, kb, j0;
+      fin_tile(a, tile, ntile_seq, &b, &q0, &kb, &j0, &nk);
+      const int64_t N = __ldg(a.kvoff + b + 1) - kb;
+      if (q0 < 0 || q0 >= a.total_q || kb < 0 || kb + N > a.total_kv || N > stride) {
+        if (threadIdx.x == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+      } else {
+        for (int i = threadIdx.x; i < 2 * Hq; i += kFinKeys) fst[i] = __ldg(ml + q0 * Hq * 2 + i);
+        cp_async_wait_prev();  // this tile's copy has landed (the next may be in flight)
+        __syncthreads();
+        const int kj = threadIdx.x;
+        if (kj < nk) {
+          const float* x = buf[cur] + kj * pitch;
+          for (int g = 0; g < a.Hkv; ++g) {
+            float sc = 0.f;
+            if (vec4) {  // 16-byte reads: the row pitch of 9 x 16 bytes spreads 8 lanes over all banks
+              for (int h = g * a.G; h < (g + 1) * a.G; h += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(x + h);
+                sc = fmaf(expf(v.x - fst[2 * h]), fst[2 * h + 1], sc);
+                sc = fmaf(expf(v.y - fst[2 * h + 2]), fst[2 * h + 3], sc);
+                sc = fmaf(expf(v.z - fst[2 * h + 4]), fst[2 * h + 5], sc);
+                sc = fmaf(expf(v.w - fst[2 * h + 6]), fst[2 * h + 7], sc);
+              }
+            } else {
+              for (int h = g * a.G; h < (g + 1) * a.G; ++h)
+                sc = fmaf(expf(x[h] - fst[2 * h]), fst[2 * h + 1], sc);
+            }
+            scores[(q0 * a.Hkv + g) * stride + j0 + kj] = sc;
+          }
+        }
+      }
+    }
+    __syncthreads();  // buffer ``cur`` is free again
+    tile = nt;
+    have = nhave;
+    cur ^= 1;
   }
-  for (int g = threadIdx.x >> 6; g < a.Hkv; g += 4) {
-    const float* x = a.logits + key * a.Hq + (int64_t)g * a.G;
-    const float* st = ml + (q0 * a.Hq + (int64_t)g * a.G) * 2;
-    float s = 0.f;
-    for (int h = 0; h < a.G; ++h) s += expf(x[h] - st[2 * h]) / st[2 * h + 1];
-    scores[(q0 * a.Hkv + g) * stride + j] = s;
-  }
+  cp_async_wait_all_groups();
 }
 
 }  // namespace hs2

@@ -23,14 +23,20 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kDecStages = 3;     // bf16 decode ring depth (2 CTAs per SM)
+constexpr int kMaxHq = 192;      // query heads the score finalize can stage
+constexpr int kSelSmemKeys = 16384;  // select: per-CTA slice kept in shared memory (64 KB)
+constexpr size_t kSpSmem = 2 * (size_t)kSpPiece * kSpRowBytes + kSpPiece * 8;  // sparse: rows + positions
 constexpr size_t kAlign = 256;
 
 struct DeviceInfo {
   bool ready = false;
+  bool cluster16 = false;  // non-portable 16-CTA clusters allowed for the select kernel
   int sms = 0;
   int* err = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
+
+size_t finalize_smem(int Hq) { return (2 * (size_t)kFinKeys * (Hq + 4) + 2 * (size_t)Hq) * sizeof(float); }
 std::mutex g_dev_mu;
 
 hs2_status device_info(DeviceInfo** out) {
@@ -48,12 +54,23 @@ hs2_status device_info(DeviceInfo** out) {
                              dec_smem) != cudaSuccess)
       return HS2_ERR_CUDA;
     if (cudaFuncSetAttribute(k_sparse_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             2 * 256 * kSpRowBytes + 256) != cudaSuccess)
+                             (int)kSpSmem) != cudaSuccess)
       return HS2_ERR_CUDA;
     if (cudaFuncSetAttribute(k_chunk_bf16<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kChStages * 2 * kChKBytes + 1024) != cudaSuccess ||
         cudaFuncSetAttribute(k_chunk_bf16<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kChStages * kChKBytes + 1024) != cudaSuccess)
+      return HS2_ERR_CUDA;
+    if (cudaFuncSetAttribute(k_select_cluster<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSelSmemKeys * 4) != cudaSuccess ||
+        cudaFuncSetAttribute(k_select_cluster<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSelSmemKeys * 4) != cudaSuccess)
+      return HS2_ERR_CUDA;
+    d.cluster16 = cudaFuncSetAttribute(k_select_cluster<16>,
+                                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    cudaGetLastError();  // a refused non-portable size is not an error
+    if (cudaFuncSetAttribute(k_finalize_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)finalize_smem(kMaxHq)) != cudaSuccess)
       return HS2_ERR_CUDA;
     d.ready = true;
   }
@@ -79,6 +96,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 hs2_status check_problem(const hs2_problem* p) {
   if (!p) return HS2_ERR_INVALID_ARG;
   if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->Hq % p->Hkv != 0) return HS2_ERR_INVALID_ARG;
+  if (p->B > 65535 || p->Hkv > 65535 || p->Hq > kMaxHq) return HS2_ERR_UNSUPPORTED;
   if (p->reserved != 0) return HS2_ERR_INVALID_ARG;
   if (p->dtype != HS2_F32 && p->dtype != HS2_BF16) return HS2_ERR_INVALID_ARG;
   if (!p->q_offsets || !p->kv_offsets) return HS2_ERR_INVALID_ARG;
@@ -173,7 +191,7 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     if (encode_kv_map(&mk, K, p) != HS2_OK || encode_kv_map(&mv, V, p) != HS2_OK) return HS2_ERR_CUDA;
     k_decode_bf16<kDecStages><<<grid, 32 * (kDecWarps + 1), kDecStages * kDecStageBytes + 1024, st>>>(mk, mv, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    k_decode_combine<bf16><<<dim3(p->B, p->Hkv), kD, 0, st>>>(a, static_cast<bf16*>(O), pl.ml);
+    k_decode_combine<bf16><<<dim3(p->B, p->Hkv, a.G), kD, 0, st>>>(a, static_cast<bf16*>(O), pl.ml);
   } else {
     const int G = a.G;
     if (G <= 1) launch_decode_f32<1>(grid, st, a);
@@ -182,11 +200,17 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     else if (G <= 8) launch_decode_f32<8>(grid, st, a);
     else launch_decode_f32<16>(grid, st, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    k_decode_combine<float><<<dim3(p->B, p->Hkv), kD, 0, st>>>(a, static_cast<float*>(O), pl.ml);
+    k_decode_combine<float><<<dim3(p->B, p->Hkv, a.G), kD, 0, st>>>(a, static_cast<float*>(O), pl.ml);
   }
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  if (p->total_kv > 0) {
-    k_finalize_scores<<<(unsigned)((p->total_kv + 63) / 64), 256, 0, st>>>(a, pl.ml, scores, stride);
+  if (p->max_kv_len > 0) {
+    const int ntile_seq = (int)((p->max_kv_len + kFinKeys - 1) / kFinKeys);
+    const int64_t ntiles = (int64_t)p->B * ntile_seq;
+    int per_sm = 1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_finalize_scores, kFinKeys, finalize_smem(p->Hq));
+    const int64_t grid = std::min<int64_t>(ntiles, (int64_t)std::max(1, per_sm) * dev.sms);
+    k_finalize_scores<<<(unsigned)grid, kFinKeys, finalize_smem(p->Hq), st>>>(a, pl.ml, scores, stride,
+                                                                               ntile_seq);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
   }
   return HS2_OK;
@@ -257,84 +281,62 @@ hs2_status run_chunk(const hs2_problem* p, const DeviceInfo& dev, const void* Q,
 // --------------------------------------------------------------------------
 // selection
 // --------------------------------------------------------------------------
-struct SelectPlan {
-  int nslices;
-  uint32_t *hist, *ticket, *prefix;
-  int32_t *krem, *cnt;
-  size_t bytes;
-};
-
-SelectPlan plan_select(int64_t rows, int64_t max_len, Carve& c) {
-  SelectPlan s{};
-  s.nslices = (int)std::max<int64_t>(1, (max_len + kSelSlice - 1) / kSelSlice);
-  const size_t before = c.used;
-  s.hist = c.take<uint32_t>((size_t)rows * kSelBins);
-  s.ticket = c.take<uint32_t>((size_t)rows);
-  s.prefix = c.take<uint32_t>((size_t)rows);
-  s.krem = c.take<int32_t>((size_t)rows);
-  s.cnt = c.take<int32_t>((size_t)rows * s.nslices * 2);
-  s.bytes = c.used - before;
-  return s;
-}
-
 // Runs the radix select over ``data`` rows and writes the ascending selection
 // to ``out``; ``count`` non-null for token rows (window, padding and count).
-hs2_status run_select(const hs2_problem* p, const DeviceInfo& dev, const SelectPlan& sp,
-                      const float* data, int64_t stride, int k, int window, int block,
-                      int32_t* out, int64_t out_stride, int32_t* count, cudaStream_t st) {
+// One cluster of CTAs per row: 16 when the rows are long and that size is
+// allowed, else 8.
+hs2_status run_select(const hs2_problem* p, const DeviceInfo& dev, const float* data,
+                      int64_t stride, int64_t max_len, int k, int window, int block, int32_t* out,
+                      int64_t out_stride, int32_t* count, cudaStream_t st) {
   const int64_t rows = p->total_q * p->Hkv;
   if (rows == 0) return HS2_OK;
-  // histogram and tickets start at zero; the last CTA of each pass cleans up after itself
-  if (cudaMemsetAsync(sp.hist, 0, (size_t)rows * kSelBins * 4, st) != cudaSuccess) return HS2_ERR_CUDA;
-  if (cudaMemsetAsync(sp.ticket, 0, (size_t)rows * 4, st) != cudaSuccess) return HS2_ERR_CUDA;
   SelectArgs a{};
   a.data = data; a.stride = stride; a.qoff = p->q_offsets; a.kvoff = p->kv_offsets;
   a.B = p->B; a.Hkv = p->Hkv; a.rows = rows; a.k = k; a.window = window; a.block = block;
-  a.nslices = sp.nslices; a.hist = sp.hist; a.ticket = sp.ticket; a.prefix = sp.prefix;
-  a.krem = sp.krem; a.cnt = sp.cnt; a.out = out; a.out_stride = out_stride; a.err = dev.err;
-  const dim3 grid((unsigned)rows, sp.nslices);
-  for (int pass = 0; pass < 3; ++pass) {
-    k_select_hist<<<grid, kSelThreads, 0, st>>>(a, pass);
-    if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  }
-  k_select_count<<<grid, kSelThreads, 0, st>>>(a);
-  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  k_select_compact<<<grid, kSelThreads, 0, st>>>(a, count);
-  return launch_status();
+  a.out = out; a.out_stride = out_stride; a.err = dev.err;
+  const int64_t len = std::max<int64_t>(1, max_len);
+  const int cs = (dev.cluster16 && len > 8 * (int64_t)kSelSmemKeys) ? 16 : 8;
+  int64_t S = (len + cs - 1) / cs;
+  S = (S + kSelChunkAlign - 1) / kSelChunkAlign * kSelChunkAlign;
+  a.slice = S;
+  a.smem_keys = S <= kSelSmemKeys ? 1 : 0;
+  if (rows * cs >= (int64_t(1) << 31)) return HS2_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * cs));
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = a.smem_keys ? (size_t)S * 4 : 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cs == 16 ? cudaLaunchKernelEx(&cfg, k_select_cluster<16>, a, count)
+                                  : cudaLaunchKernelEx(&cfg, k_select_cluster<8>, a, count);
+  return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 
 // --------------------------------------------------------------------------
-// sparse attention plan
+// sparse attention: one cluster of kSpCluster CTAs per (query, KV group) row
 // --------------------------------------------------------------------------
-struct SparsePlan {
-  int chunk, nchunk;
-  float *pm, *pl, *po;
-  uint32_t* ticket;
-  size_t bytes;
-};
-
-SparsePlan plan_sparse(const hs2_problem* p, const DeviceInfo& dev, int idx_stride, void* ws) {
-  SparsePlan s{};
-  const int64_t rows = std::max<int64_t>(1, p->total_q * p->Hkv);
-  const int64_t target = (int64_t)dev.sms * 2;
-  int64_t ch = (rows * idx_stride + target - 1) / target;
-  ch = (ch + 15) / 16 * 16;
-  s.chunk = (int)std::min<int64_t>(256, std::max<int64_t>(16, ch));
-  s.nchunk = (int)std::max<int64_t>(1, (idx_stride + s.chunk - 1) / s.chunk);
-  const int G = p->Hq / p->Hkv;
-  Carve c(ws);
-  const size_t slots = (size_t)rows * s.nchunk * kSpWarps * G;
-  s.pm = c.take<float>(slots);
-  s.pl = c.take<float>(slots);
-  s.po = c.take<float>(slots * kD);
-  s.ticket = c.take<uint32_t>((size_t)rows);
-  s.bytes = c.used;
-  return s;
-}
-
-template <int GP>
-void launch_sparse_f32(dim3 grid, cudaStream_t st, const SparseArgs& a) {
-  k_sparse_f32<GP><<<grid, 32 * kSpWarps, 0, st>>>(a);
+template <typename Kern>
+cudaError_t launch_cluster(Kern kern, unsigned ctas, unsigned threads, size_t smem, int cs,
+                           cudaStream_t st, const SparseArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 hs2_status check_ws(void* ws, size_t have, size_t need) {
@@ -386,15 +388,15 @@ hs2_status hs2_topk_workspace_size(const hs2_problem* p, int32_t k, int32_t wind
   if (!bytes || k < 1 || window < 1) return HS2_ERR_INVALID_ARG;
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
-  Carve c(nullptr);
-  plan_select(p->total_q * p->Hkv, p->max_kv_len, c);
-  *bytes = c.used;
+  *bytes = 0;  // the selection keeps all of its state on chip
   return HS2_OK;
 }
 
 hs2_status hs2_topk_select(const hs2_problem* p, const float* scores, int64_t score_stride, int32_t k,
                            int32_t window, int32_t* idx, int32_t* count, void* workspace,
                            size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
   if (!scores || !idx || !count || k < 1 || window < 1) return HS2_ERR_INVALID_ARG;
@@ -402,13 +404,8 @@ hs2_status hs2_topk_select(const hs2_problem* p, const float* scores, int64_t sc
   if (!aligned16(scores) || score_stride < std::max<int64_t>(1, p->max_kv_len)) return HS2_ERR_INVALID_ARG;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != HS2_OK) return s;
-  Carve c(nullptr);
-  plan_select(p->total_q * p->Hkv, p->max_kv_len, c);
-  if ((s = check_ws(workspace, workspace_bytes, c.used)) != HS2_OK) return s;
-  Carve w(workspace);
-  const SelectPlan sp = plan_select(p->total_q * p->Hkv, p->max_kv_len, w);
-  return run_select(p, *dev, sp, scores, score_stride, k, window, 0, idx, (int64_t)k + window, count,
-                    static_cast<cudaStream_t>(stream));
+  return run_select(p, *dev, scores, score_stride, p->max_kv_len, k, window, 0, idx,
+                    (int64_t)k + window, count, static_cast<cudaStream_t>(stream));
 }
 
 hs2_status hs2_block_select_workspace_size(const hs2_problem* p, int32_t n_blocks, int32_t block,
@@ -421,7 +418,6 @@ hs2_status hs2_block_select_workspace_size(const hs2_problem* p, int32_t n_block
   Carve c(nullptr);
   c.take<float>((size_t)rows * nb);
   c.take<int32_t>((size_t)rows * n_blocks);
-  plan_select(rows, nb, c);
   *bytes = c.used;
   return HS2_OK;
 }
@@ -446,11 +442,10 @@ hs2_status hs2_block_select(const hs2_problem* p, const float* scores, int64_t s
   Carve w(workspace);
   float* bmax = w.take<float>((size_t)rows * nb);
   int32_t* bsel = w.take<int32_t>((size_t)rows * n_blocks);
-  const SelectPlan sp = plan_select(rows, nb, w);
   k_block_max<<<dim3((unsigned)rows, (unsigned)((nb + 7) / 8)), 256, 0, st>>>(
       scores, score_stride, p->q_offsets, p->kv_offsets, p->B, p->Hkv, block, window, bmax, nb, dev->err);
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  if ((s = run_select(p, *dev, sp, bmax, nb, n_blocks, window, block, bsel, n_blocks, nullptr, st)) != HS2_OK)
+  if ((s = run_select(p, *dev, bmax, nb, nb, n_blocks, window, block, bsel, n_blocks, nullptr, st)) != HS2_OK)
     return s;
   k_block_expand<<<(unsigned)rows, 256, 0, st>>>(bsel, n_blocks, p->q_offsets, p->kv_offsets, p->B,
                                                  p->Hkv, block, window, idx,
@@ -462,48 +457,44 @@ hs2_status hs2_sparse_attn_workspace_size(const hs2_problem* p, int32_t idx_stri
   if (!bytes || idx_stride < 1) return HS2_ERR_INVALID_ARG;
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
-  DeviceInfo* dev;
-  if ((s = device_info(&dev)) != HS2_OK) return s;
-  *bytes = plan_sparse(p, *dev, idx_stride, nullptr).bytes;
+  *bytes = 0;  // the partials of a row are merged on chip, inside its cluster
   return HS2_OK;
 }
 
 hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K, const void* V,
                            const int32_t* idx, const int32_t* count, int32_t idx_stride, void* O_l,
                            void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
   if (!Q_l || !K || !V || !idx || !count || !O_l || idx_stride < 1) return HS2_ERR_INVALID_ARG;
   if (!aligned16(Q_l) || !aligned16(K) || !aligned16(V) || !aligned16(O_l)) return HS2_ERR_INVALID_ARG;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != HS2_OK) return s;
-  const SparsePlan sp0 = plan_sparse(p, *dev, idx_stride, nullptr);
-  if ((s = check_ws(workspace, workspace_bytes, sp0.bytes)) != HS2_OK) return s;
   const int64_t rows = p->total_q * p->Hkv;
   if (rows == 0) return HS2_OK;
+  if (rows * kSpCluster >= (int64_t(1) << 31)) return HS2_ERR_UNSUPPORTED;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const SparsePlan sp = plan_sparse(p, *dev, idx_stride, workspace);
-  if (cudaMemsetAsync(sp.ticket, 0, (size_t)rows * 4, st) != cudaSuccess) return HS2_ERR_CUDA;
   SparseArgs a{};
   a.Q = Q_l; a.K = K; a.V = V; a.idx = idx; a.count = count; a.idx_stride = idx_stride;
   a.qoff = p->q_offsets; a.kvoff = p->kv_offsets;
   a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = p->Hq / p->Hkv;
   a.total_q = p->total_q; a.total_kv = p->total_kv; a.scale = p->scale;
-  a.chunk = sp.chunk; a.nchunk = sp.nchunk; a.pm = sp.pm; a.pl = sp.pl; a.po = sp.po;
-  a.ticket = sp.ticket; a.O = O_l; a.err = dev->err;
-  const dim3 grid((unsigned)rows, sp.nchunk);
+  a.O = O_l; a.err = dev->err;
+  const unsigned ctas = (unsigned)(rows * kSpCluster);
+  cudaError_t e;
   if (p->dtype == HS2_BF16) {
-    const size_t smem = 2 * (size_t)sp.chunk * kSpRowBytes + sp.chunk;
-    k_sparse_bf16<<<grid, 32 * kSpWarps, smem, st>>>(a);
+    e = launch_cluster(k_sparse_bf16, ctas, 32 * kSpWarps, kSpSmem, kSpCluster, st, a);
   } else {
     const int G = a.G;
-    if (G <= 1) launch_sparse_f32<1>(grid, st, a);
-    else if (G <= 2) launch_sparse_f32<2>(grid, st, a);
-    else if (G <= 4) launch_sparse_f32<4>(grid, st, a);
-    else if (G <= 8) launch_sparse_f32<8>(grid, st, a);
-    else launch_sparse_f32<16>(grid, st, a);
+    if (G <= 1) e = launch_cluster(k_sparse_f32<1>, ctas, 32 * kSpWarps, 0, kSpCluster, st, a);
+    else if (G <= 2) e = launch_cluster(k_sparse_f32<2>, ctas, 32 * kSpWarps, 0, kSpCluster, st, a);
+    else if (G <= 4) e = launch_cluster(k_sparse_f32<4>, ctas, 32 * kSpWarps, 0, kSpCluster, st, a);
+    else if (G <= 8) e = launch_cluster(k_sparse_f32<8>, ctas, 32 * kSpWarps, 0, kSpCluster, st, a);
+    else e = launch_cluster(k_sparse_f32<16>, ctas, 32 * kSpWarps, 0, kSpCluster, st, a);
   }
-  return launch_status();
+  return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 
 hs2_status hs2_get_last_device_error(void* stream) {

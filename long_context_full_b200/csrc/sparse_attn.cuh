@@ -7,21 +7,29 @@
 // and selection) and "Token-Level Selection and Unified Local Access" (local and
 // global tokens come from the one shared cache, in a single sparse computation).
 //
-// Grid (chunks, rows): the index list of a row (<= k + window entries) is cut
-// into chunks of ``chunk`` indices so that every SM has work even at batch 1.
-// Each CTA gathers its rows of K and V into shared memory with bulk copies (the
-// TMA engine, one 256-byte copy per row and tensor), computes per-warp online
-// softmax partials on the tensor cores, and the last CTA of the row (atomic
-// ticket, no spinning) merges the partials into O.
+// One thread-block cluster of kSpCluster CTAs per (query, KV group) row: CTA c
+// takes the c-th share of the row's index list, gathers those K/V rows into
+// shared memory with 16-byte cp.async copies (rows are 256 bytes: too small for
+// efficient TMA requests), runs an online softmax per warp (tensor cores for
+// bf16), folds its warps into one partial, and the cluster merges the partials
+// through distributed shared memory - CTA c finishing the heads h = c mod
+// kSpCluster after a single cluster barrier.  No workspace, no global round
+// trip, no atomics.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "ptx.cuh"
 
 namespace hs2 {
 
+namespace cg = cooperative_groups;
+
 constexpr int kSpWarps = 4;
+constexpr int kSpCluster = 8;
 constexpr int kSpRowBytes = 272;  // 256-byte bf16 row + 16 bytes: conflict-free ldmatrix
+constexpr int kSpPiece = 160;     // gathered rows staged per round (10 slices of 16)
 
 struct SparseArgs {
   const void* Q;        // [total_q, Hq, D], this layer's queries
@@ -35,48 +43,18 @@ struct SparseArgs {
   int B, Hq, Hkv, G;
   int64_t total_q, total_kv;
   float scale;
-  int chunk, nchunk;    // indices per CTA, grid.y (grid.x = rows)
-  float* pm;            // [rows, nchunk, kSpWarps, G]
-  float* pl;
-  float* po;            // [rows, nchunk, kSpWarps, G, D]
-  uint32_t* ticket;     // [rows], zero on entry
   void* O;              // [total_q, Hq, D]
   int* err;
 };
 
-// Last CTA of a row: merge the (nchr x warps) partials into O.  D threads.
-template <typename OT>
-__device__ void sparse_merge(const SparseArgs& a, int64_t r, int nchr) {
-  const int64_t qi = r / a.Hkv;
-  const int g = (int)(r % a.Hkv);
-  const int d = threadIdx.x;
-  if (d >= kD) return;
-  OT* O = static_cast<OT*>(a.O);
-  for (int hl = 0; hl < a.G; ++hl) {
-    float M = -INFINITY;
-    for (int c = 0; c < nchr; ++c)
-      for (int w = 0; w < kSpWarps; ++w)
-        M = fmaxf(M, __ldcg(a.pm + ((r * a.nchunk + c) * kSpWarps + w) * a.G + hl));
-    float L = 0.f, acc = 0.f;
-    for (int c = 0; c < nchr; ++c)
-      for (int w = 0; w < kSpWarps; ++w) {
-        const int64_t pi = ((r * a.nchunk + c) * kSpWarps + w) * a.G + hl;
-        const float wt = exp_shift(__ldcg(a.pm + pi), M);
-        L = fmaf(__ldcg(a.pl + pi), wt, L);
-        acc = fmaf(__ldcg(a.po + pi * kD + d), wt, acc);
-      }
-    O[(qi * a.Hq + (int64_t)g * a.G + hl) * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
-  }
-}
-
-// Common prologue: row geometry and this CTA's index range; false = no work.
+// This CTA's share of a row: indices [j0, j0 + n) of the row's list.
 struct SpRow {
   int64_t r, qi, kv_start, t;
-  int g, c, cnt, nchr, j0, n;
+  int g, cnt, j0, n;
 };
-__device__ __forceinline__ bool sparse_row(const SparseArgs& a, SpRow& s) {
-  s.r = blockIdx.x;
-  s.c = blockIdx.y;
+__device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int cs) {
+  SpRow s;
+  s.r = blockIdx.x / cs;
   s.qi = s.r / a.Hkv;
   s.g = (int)(s.r % a.Hkv);
   const QueryRow q = query_row(a.qoff, a.kvoff, a.B, s.qi);
@@ -84,91 +62,101 @@ __device__ __forceinline__ bool sparse_row(const SparseArgs& a, SpRow& s) {
   s.t = q.t;
   int cnt = __ldg(a.count + s.r);
   if (cnt < 0 || cnt > a.idx_stride) {
-    if (threadIdx.x == 0 && s.c == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+    if (threadIdx.x == 0 && rank == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
     cnt = cnt < 0 ? 0 : a.idx_stride;
   }
   s.cnt = cnt;
-  s.nchr = cnt > 0 ? (cnt + a.chunk - 1) / a.chunk : 1;
-  if (s.c >= s.nchr) return false;
-  s.j0 = s.c * a.chunk;
-  const int j1 = s.j0 + a.chunk < cnt ? s.j0 + a.chunk : cnt;
-  s.n = j1 > s.j0 ? j1 - s.j0 : 0;
-  return true;
+  int per = (cnt + cs - 1) / cs;
+  per = (per + 15) / 16 * 16;
+  s.j0 = rank * per;
+  s.n = cnt - s.j0 < 0 ? 0 : (cnt - s.j0 < per ? cnt - s.j0 : per);
+  return s;
 }
 
-// Position of index i of the row, or -1 (recorded) if outside 0..t.
-__device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& s, int i) {
+// Cache position of list entry i of the CTA's share, or -1 (recorded) if
+// outside 0..t.
+__device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& s, int i,
+                                              bool record) {
   const int64_t pos = __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
   if (pos < 0 || pos > s.t || s.kv_start + pos >= a.total_kv) {
-    record_error(a.err, HS2_ERR_DEVICE_INPUT);
+    if (record) record_error(a.err, HS2_ERR_DEVICE_INPUT);
     return -1;
   }
   return pos;
 }
 
-template <typename OT>
-__device__ __forceinline__ void sparse_finish(const SparseArgs& a, const SpRow& s) {
-  __shared__ int is_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) is_last = (atomicAdd(a.ticket + s.r, 1u) == (uint32_t)(s.nchr - 1));
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  sparse_merge<OT>(a, s.r, s.nchr);
-  if (threadIdx.x == 0) a.ticket[s.r] = 0u;
+// Partials received by the CTA that finishes a head: one slot per source CTA
+// and per owned head (heads h with h % cs == rank; at most kSpOwned of them).
+constexpr int kSpOwned = 2;
+struct SpRecv {
+  float m[kSpCluster][kSpOwned];
+  float l[kSpCluster][kSpOwned];
+  float o[kSpCluster][kSpOwned][kD];
+};
+
+// Cluster merge.  Each CTA folds its warps' partials (wm/wl [kSpWarps][GMAX],
+// wo [kSpWarps][GMAX][D]) into one partial per head and pushes it into the
+// shared memory of CTA h % cs (distributed shared memory stores); one cluster
+// barrier makes them visible, and each CTA finishes its own heads from local
+// memory.  Nothing is read remotely after the barrier, so it is the only one.
+// D threads.
+template <typename OT, int GMAX>
+__device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_t qi, int g,
+                                                     cg::cluster_group& cl, int rank, int cs,
+                                                     const float* wm, const float* wl,
+                                                     const float* wo, SpRecv& recv) {
+  const int d = threadIdx.x;
+  for (int h = 0; h < a.G; ++h) {
+    float M = -INFINITY;
+    for (int w = 0; w < kSpWarps; ++w) M = fmaxf(M, wm[w * GMAX + h]);
+    float L = 0.f, acc = 0.f;
+    for (int w = 0; w < kSpWarps; ++w) {
+      const float wt = exp_shift(wm[w * GMAX + h], M);
+      L = fmaf(wl[w * GMAX + h], wt, L);
+      acc = fmaf(wo[(w * GMAX + h) * kD + d], wt, acc);
+    }
+    SpRecv* dst = cl.map_shared_rank(&recv, h % cs);
+    const int slot = h / cs;
+    dst->o[rank][slot][d] = acc;
+    if (d == 0) {
+      dst->m[rank][slot] = M;
+      dst->l[rank][slot] = L;
+    }
+  }
+  cl.sync();
+  OT* O = static_cast<OT*>(a.O);
+  for (int h = rank; h < a.G; h += cs) {
+    const int slot = h / cs;
+    float M = -INFINITY;
+    for (int c = 0; c < cs; ++c) M = fmaxf(M, recv.m[c][slot]);
+    float L = 0.f, acc = 0.f;
+    for (int c = 0; c < cs; ++c) {
+      const float wt = exp_shift(recv.m[c][slot], M);
+      L = fmaf(recv.l[c][slot], wt, L);
+      acc = fmaf(recv.o[c][slot][d], wt, acc);
+    }
+    O[(qi * a.Hq + (int64_t)g * a.G + h) * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
+  }
 }
 
 // ----------------------------------------------------------------------------
-// bf16: gathered rows staged by bulk copies, tensor-core S^T = K Q^T and
-// O^T += V^T P^T per 16-key slice (same fragment scheme as the decode pass).
+// bf16: tensor-core S^T = K Q^T and O^T += V^T P^T per 16-key slice, the same
+// fragment scheme as the decode pass (P^T by one movmatrix transpose).
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_constant__ SparseArgs a) {
   extern __shared__ __align__(128) uint8_t sp_smem[];
-  __shared__ __align__(8) uint64_t bar;
-  SpRow s;
-  if (!sparse_row(a, s)) return;
+  __shared__ float wm[kSpWarps * 8], wl[kSpWarps * 8];
+  __shared__ float wo[kSpWarps * 8 * kD];
+  __shared__ SpRecv recv;
+  cg::cluster_group cl = cg::this_cluster();
+  const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const SpRow s = sparse_row(a, rank, cs);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* sK = sp_smem;
-  uint8_t* sV = sp_smem + (size_t)a.chunk * kSpRowBytes;
-  int8_t* valid = reinterpret_cast<int8_t*>(sp_smem + 2 * (size_t)a.chunk * kSpRowBytes);
+  uint8_t* sV = sp_smem + (size_t)kSpPiece * kSpRowBytes;
+  int64_t* spos = reinterpret_cast<int64_t*>(sp_smem + 2 * (size_t)kSpPiece * kSpRowBytes);
   const bf16* K = static_cast<const bf16*>(a.K);
   const bf16* V = static_cast<const bf16*>(a.V);
-
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, blockDim.x);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  // gather: thread i copies rows i, i + 128, ...
-  uint32_t bytes = 0;
-  for (int i = threadIdx.x; i < s.n; i += blockDim.x) {
-    const int64_t pos = sparse_pos(a, s, i);
-    valid[i] = pos >= 0;
-    if (pos >= 0) bytes += 2 * kD * sizeof(bf16);
-  }
-  mbar_arrive_expect_tx(&bar, bytes);
-  for (int i = threadIdx.x; i < s.n; i += blockDim.x) {
-    if (!valid[i]) continue;
-    const int64_t pos = __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
-    const int64_t row = (s.kv_start + pos) * a.Hkv + s.g;
-    bulk_g2s(sK + (size_t)i * kSpRowBytes, K + row * kD, kD * sizeof(bf16), &bar);
-    bulk_g2s(sV + (size_t)i * kSpRowBytes, V + row * kD, kD * sizeof(bf16), &bar);
-  }
-  // rows past n or invalid must not feed NaNs into the MMAs: zero them
-  const int ntile = (s.n + 15) / 16;
-  for (int i = threadIdx.x; i < ntile * 16; i += blockDim.x) {
-    if (i < s.n && valid[i]) continue;
-    uint4* zk = reinterpret_cast<uint4*>(sK + (size_t)i * kSpRowBytes);
-    uint4* zv = reinterpret_cast<uint4*>(sV + (size_t)i * kSpRowBytes);
-    for (int c = 0; c < 16; ++c) zk[c] = zv[c] = make_uint4(0u, 0u, 0u, 0u);
-  }
-  const bool landed = mbar_wait(&bar, 0);
-  if (!landed) {
-    record_error(a.err, HS2_ERR_TIMEOUT);
-    mbar_wait(&bar, 0);  // give copies still in flight a second bounded chance to land
-  }
-  __syncthreads();
 
   const int r = lane >> 2, qd = lane & 3;
   const int h0 = 2 * qd, h1 = 2 * qd + 1;
@@ -190,85 +178,108 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   const uint32_t skb = smem_u32(sK), svb = smem_u32(sV);
-  for (int st = warp; landed && st < ntile; st += kSpWarps) {
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
-    {
-      const int row = st * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+
+  for (int p0 = 0; p0 < s.n; p0 += kSpPiece) {
+    const int pn = s.n - p0 < kSpPiece ? s.n - p0 : kSpPiece;
+    const int ntile = (pn + 15) / 16;
+    // the piece's cache rows (-1: past the list or invalid), read once
+    for (int row = threadIdx.x; row < ntile * 16; row += blockDim.x)
+      spos[row] = row < pn ? sparse_pos(a, s, p0 + row, true) : -1;
+    __syncthreads();
+    // gather: 16-byte cp.async per (row, chunk), 16 chunks of K and 16 of V per
+    // row; rows past pn or with an invalid index are zero-filled (no read)
+    for (int i = threadIdx.x; i < ntile * 16 * 32; i += blockDim.x) {
+      const int row = i >> 5, ch = i & 31, c16 = ch & 15;
+      const int64_t pos = spos[row];
+      const bool ok = pos >= 0;
+      const bf16* base = ch < 16 ? K : V;
+      const bf16* src = ok ? base + ((s.kv_start + pos) * a.Hkv + s.g) * kD + c16 * 8 : base;
+      uint8_t* dst = (ch < 16 ? sK : sV) + (size_t)row * kSpRowBytes + c16 * 16;
+      cp_async16(dst, src, ok ? 16 : 0);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    for (int st = warp; st < ntile; st += kSpWarps) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int row = st * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int chunk = kk * 2 + (lane >> 4);
+        for (int kk = 0; kk < 8; ++kk) {
+          const int chunk = kk * 2 + (lane >> 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a0, a1, a2, a3, skb + row * kSpRowBytes + chunk * 16);
+          mma_bf16(c, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+        }
+      }
+      const int ilo = st * 16 + r, ihi = ilo + 8;
+      const bool vlo = spos[ilo] >= 0, vhi = spos[ihi] >= 0;
+      const float x0 = vlo ? c[0] * a.scale : NEG, x1 = vlo ? c[1] * a.scale : NEG;
+      const float x2 = vhi ? c[2] * a.scale : NEG, x3 = vhi ? c[3] * a.scale : NEG;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = (mn0 == NEG) ? 1.f : exp_shift(m0, mn0);
+      const float al1 = (mn1 == NEG) ? 1.f : exp_shift(m1, mn1);
+      const float p0v = exp_shift(x0, mn0), p1v = exp_shift(x1, mn1);
+      const float p2v = exp_shift(x2, mn0), p3v = exp_shift(x3, mn1);
+      l0 = l0 * al0 + (p0v + p2v);
+      l1 = l1 * al1 + (p1v + p3v);
+      m0 = mn0;
+      m1 = mn1;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[i][0] *= al0; o[i][1] *= al1; o[i][2] *= al0; o[i][3] *= al1;
+      }
+      const uint32_t b0 = movmatrix_t(pack_bf16(p0v, p1v));
+      const uint32_t b1 = movmatrix_t(pack_bf16(p2v, p3v));
+      const int row = st * 16 + ((lane >> 4) & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int chunk = mt * 2 + ((lane >> 3) & 1);
         uint32_t a0, a1, a2, a3;
-        ldsm_x4(a0, a1, a2, a3, skb + row * kSpRowBytes + chunk * 16);
-        mma_bf16(c, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+        ldsm_x4_t(a0, a1, a2, a3, svb + row * kSpRowBytes + chunk * 16);
+        mma_bf16(o[mt], a0, a1, a2, a3, b0, b1);
       }
     }
-    const int ilo = st * 16 + r, ihi = ilo + 8;
-    const bool vlo = ilo < s.n && valid[ilo], vhi = ihi < s.n && valid[ihi];
-    const float x0 = vlo ? c[0] * a.scale : NEG, x1 = vlo ? c[1] * a.scale : NEG;
-    const float x2 = vhi ? c[2] * a.scale : NEG, x3 = vhi ? c[3] * a.scale : NEG;
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float al0 = (mn0 == NEG) ? 1.f : exp_shift(m0, mn0);
-    const float al1 = (mn1 == NEG) ? 1.f : exp_shift(m1, mn1);
-    const float p0 = exp_shift(x0, mn0), p1 = exp_shift(x1, mn1);
-    const float p2 = exp_shift(x2, mn0), p3 = exp_shift(x3, mn1);
-    l0 = l0 * al0 + (p0 + p2);
-    l1 = l1 * al1 + (p1 + p3);
-    m0 = mn0;
-    m1 = mn1;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      o[i][0] *= al0; o[i][1] *= al1; o[i][2] *= al0; o[i][3] *= al1;
-    }
-    const uint32_t b0 = movmatrix_t(pack_bf16(p0, p1));
-    const uint32_t b1 = movmatrix_t(pack_bf16(p2, p3));
-    const int row = st * 16 + ((lane >> 4) & 1) * 8 + (lane & 7);
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      const int chunk = mt * 2 + ((lane >> 3) & 1);
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4_t(a0, a1, a2, a3, svb + row * kSpRowBytes + chunk * 16);
-      mma_bf16(o[mt], a0, a1, a2, a3, b0, b1);
-    }
+    __syncthreads();  // the next piece overwrites the staged rows
   }
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, off);
     l1 += __shfl_xor_sync(0xffffffffu, l1, off);
   }
-  const int64_t base = ((s.r * a.nchunk + s.c) * kSpWarps + warp) * a.G;
   if (r == 0) {
-    if (h0 < a.G) { a.pm[base + h0] = m0; a.pl[base + h0] = l0; }
-    if (h1 < a.G) { a.pm[base + h1] = m1; a.pl[base + h1] = l1; }
+    wm[warp * 8 + h0] = m0; wl[warp * 8 + h0] = l0;
+    wm[warp * 8 + h1] = m1; wl[warp * 8 + h1] = l1;
   }
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
     const int d = mt * 16 + r;
-    if (h0 < a.G) {
-      a.po[(base + h0) * kD + d] = o[mt][0];
-      a.po[(base + h0) * kD + d + 8] = o[mt][2];
-    }
-    if (h1 < a.G) {
-      a.po[(base + h1) * kD + d] = o[mt][1];
-      a.po[(base + h1) * kD + d + 8] = o[mt][3];
-    }
+    wo[(warp * 8 + h0) * kD + d] = o[mt][0];
+    wo[(warp * 8 + h0) * kD + d + 8] = o[mt][2];
+    wo[(warp * 8 + h1) * kD + d] = o[mt][1];
+    wo[(warp * 8 + h1) * kD + d + 8] = o[mt][3];
   }
-  sparse_finish<bf16>(a, s);
+  __syncthreads();
+  sparse_cluster_merge<bf16, 8>(a, s.qi, s.g, cl, rank, cs, wm, wl, wo, recv);
 }
 
 // ----------------------------------------------------------------------------
-// float32 on the CUDA cores: each warp takes every 4th index of the chunk and
-// reads its K/V rows directly (lane i holds dims 4i..4i+3).
+// float32 on the CUDA cores: each warp takes every 4th index of the CTA's share
+// and reads its K/V rows directly (lane i holds dims 4i..4i+3).
 // ----------------------------------------------------------------------------
 template <int GP>
 __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_f32(const __grid_constant__ SparseArgs a) {
-  SpRow s;
-  if (!sparse_row(a, s)) return;
+  __shared__ float wm[kSpWarps * GP], wl[kSpWarps * GP];
+  __shared__ float wo[kSpWarps * GP * kD];
+  __shared__ SpRecv recv;
+  cg::cluster_group cl = cg::this_cluster();
+  const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const SpRow s = sparse_row(a, rank, cs);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* Q = static_cast<const float*>(a.Q);
   const float* K = static_cast<const float*>(a.K);
@@ -284,8 +295,8 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_f32(const __grid_const
     l[h] = 0.f;
   }
   for (int i = warp; i < s.n; i += kSpWarps) {
-    const int64_t pos = sparse_pos(a, s, i);
-    if (pos < 0) continue;
+    const int64_t pos = sparse_pos(a, s, i, lane == 0);
+    if (pos < 0) continue;  // the CUDA-core path serves float32 checks, not speed
     const int64_t row = (s.kv_start + pos) * a.Hkv + s.g;
     const float4 kv = *reinterpret_cast<const float4*>(K + row * kD + lane * 4);
     const float4 vv = *reinterpret_cast<const float4*>(V + row * kD + lane * 4);
@@ -308,14 +319,13 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_f32(const __grid_const
       m[h] = mn;
     }
   }
-  const int64_t base = ((s.r * a.nchunk + s.c) * kSpWarps + warp) * a.G;
 #pragma unroll
   for (int h = 0; h < GP; ++h) {
-    if (h >= a.G) break;
-    if (lane == 0) { a.pm[base + h] = m[h]; a.pl[base + h] = l[h]; }
-    *reinterpret_cast<float4*>(a.po + (base + h) * kD + lane * 4) = o[h];
+    if (lane == 0) { wm[warp * GP + h] = m[h]; wl[warp * GP + h] = l[h]; }
+    *reinterpret_cast<float4*>(wo + (warp * GP + h) * kD + lane * 4) = o[h];
   }
-  sparse_finish<float>(a, s);
+  __syncthreads();
+  sparse_cluster_merge<float, GP>(a, s.qi, s.g, cl, rank, cs, wm, wl, wo, recv);
 }
 
 }  // namespace hs2

@@ -136,12 +136,14 @@ def check_index_sets(gidx, gcnt, oidx, ocnt, oscores, t, k, window, what):
 
 
 def gpu_select_on(scores_rows: np.ndarray, ts, k=1024, window=128, block_mode=False,
-                  n_blocks=16, block=64):
+                  n_blocks=16, block=64, stride=None):
     """Runs the GPU selection on given float32 score rows (one query row per
-    sequence, Hkv = 1).  ts: position t of each row.  Returns (idx, count)."""
+    sequence, Hkv = 1).  ts: position t of each row; stride: row stride of the
+    score buffer (default: the row length rounded up to 4).  Returns (idx, count)."""
     R = len(ts)
     kv_lens = np.asarray(ts, np.int64) + 1
-    stride = max(1, (scores_rows.shape[1] + 3) // 4 * 4)
+    if stride is None:
+        stride = max(1, (scores_rows.shape[1] + 3) // 4 * 4)
     S = np.zeros((R, stride), np.float32)
     S[:, :scores_rows.shape[1]] = scores_rows
     qo = torch.arange(R + 1, dtype=torch.int64).cuda()

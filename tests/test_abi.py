@@ -85,13 +85,15 @@ def test_null_problem_and_bad_call_arguments(lib):
                                     None, 0, None) == hs2.HS2_ERR_INVALID_ARG
 
 
-def test_topk_workspace_size_formula(lib):
-    # histogram (2048 x 4 B) + ticket + prefix + krem + per-slice counts, each 256-B rounded
+def test_workspace_sizes(lib):
+    """Selection and sparse layers keep their state on chip; block selection
+    needs the block maxima and the chosen block ids (each 256-byte rounded)."""
     p = _problem(total_q=3, B=3, max_kv_len=10000, total_kv=20000)
-    n = ctypes.c_size_t(0)
+    n = ctypes.c_size_t(123)
     assert lib.hs2_topk_workspace_size(ctypes.byref(p), 1024, 128, ctypes.byref(n)) == 0
+    assert n.value == 0
+    assert lib.hs2_block_select_workspace_size(ctypes.byref(p), 16, 64, 128, ctypes.byref(n)) == 0
     rows = 3 * 2
     rnd = lambda b: (b + 255) // 256 * 256
-    slices = (10000 + 4095) // 4096
-    want = rnd(rows * 2048 * 4) + 3 * rnd(rows * 4) + rnd(rows * slices * 2 * 4)
-    assert n.value == want
+    nb = (10000 + 63) // 64
+    assert n.value == rnd(rows * nb * 4) + rnd(rows * 16 * 4)

@@ -137,6 +137,64 @@ def test_select_edge_positions(t):
     assert int(cnt[0]) == oc and np.array_equal(idx[0], oi)
 
 
+def test_select_many_rows():
+    """Many rows (clusters run in several waves); a row's result does not
+    depend on the rows launched with it."""
+    rng = np.random.default_rng(17)
+    R, n = 1400, 3000
+    S = rng.integers(0, 40, (R, n)).astype(np.float32)
+    ts = list(rng.integers(1100, n, R))
+    idx, cnt = gpu_select_on(S, ts)
+    for r in range(0, R, 7):
+        oi, oc = oracle.topk_select(S[r], ts[r])
+        assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
+    # the same rows in a small batch give the same result
+    sub = list(range(0, 60))
+    i2, c2 = gpu_select_on(S[sub], [ts[r] for r in sub])
+    assert np.array_equal(i2, idx[sub]) and np.array_equal(c2, cnt[sub])
+
+
+def test_select_long_rows_wide_slices():
+    """Long rows with a large tie block straddling the threshold."""
+    rng = np.random.default_rng(23)
+    R, n = 40, 100000
+    S = rng.random((R, n)).astype(np.float32)
+    S[:, ::7] = np.float32(0.999)  # a tie block straddling the threshold
+    ts = [n - 1 - 37 * r for r in range(R)]
+    idx, cnt = gpu_select_on(S, ts)
+    for r in range(R):
+        oi, oc = oracle.topk_select(S[r], ts[r])
+        assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
+
+
+def test_select_rows_longer_than_shared_memory():
+    """Rows whose per-CTA slices do not fit in shared memory (re-read from
+    global memory on every pass)."""
+    rng = np.random.default_rng(29)
+    n = 600000
+    S = rng.standard_normal((2, n)).astype(np.float32)
+    S[1, rng.choice(n, 5000, replace=False)] = np.float32(2.5)
+    ts = [n - 1, n - 1000]
+    idx, cnt = gpu_select_on(S, ts)
+    for r in range(2):
+        oi, oc = oracle.topk_select(S[r], ts[r])
+        assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
+
+
+@pytest.mark.parametrize("stride_extra", [1, 2, 3, 37])
+def test_select_unaligned_stride(stride_extra):
+    """Score rows whose stride is not a multiple of 4 floats (the C ABI allows
+    any stride >= the longest sequence)."""
+    rng = np.random.default_rng(stride_extra)
+    n = 9000
+    S = rng.integers(0, 30, (3, n)).astype(np.float32)
+    ts = [n - 1, n - 500, 4000]
+    idx, cnt = gpu_select_on(S, ts, stride=n + stride_extra)
+    for r in range(3):
+        oi, oc = oracle.topk_select(S[r], ts[r])
+        assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
+
+
 def test_block_select_bit_exact():
     S = _select_rows()
     ts = [19999, 19999, 15000, 19999, 19999, 12345, 19999]
@@ -194,8 +252,11 @@ def test_device_input_errors_are_reported():
 
 def test_host_checks_launch_nothing():
     w = synth.make_workload("chk", 91, "bf16", 8, 1, 128, [500], [1], 1)
-    run = GpuRun(w)
+    run = GpuRun(w, select="block")
+    before = run.step.idx.clone()
     with pytest.raises(hs2.HS2Error) as e:
-        hs2.hs2_topk_select(run.step.problem, run.step.scores, run.step.stride, 1024, 128,
-                            run.step.idx, run.step.count, None)
+        hs2.hs2_block_select(run.step.problem, run.step.scores, run.step.stride, 16, 64, 128,
+                             run.step.idx, run.step.count, None)
     assert e.value.status == hs2.HS2_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.equal(before, run.step.idx)
