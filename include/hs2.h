@@ -45,8 +45,8 @@
  * Ownership.  The caller owns every buffer, including the workspace.  The
  *   library allocates no memory, never synchronises (except
  *   hs2_get_last_device_error) and launches only on ``stream``
- *   (a cudaStream_t; NULL is the legacy default stream).  Calls may be captured
- *   in a CUDA graph.  Calls that use the same workspace must not overlap.
+ *   (a cudaStream_t; NULL is the legacy default stream).  Calls that use the
+ *   same workspace must not overlap.
  * Workspace.  Query the size with the matching *_workspace_size call; pass at
  *   least that many bytes, 256-byte aligned.  Its contents on entry do not
  *   matter; on return they are unspecified.
@@ -177,6 +177,34 @@ hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K,
                            const void* V, const int32_t* idx, const int32_t* count,
                            int32_t idx_stride, void* O_l, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * hs2_block_select_noalloc - hs2_block_select for callers that cannot give
+ * the library device memory (the pages have no counterpart: this is a
+ * deployment convenience, not part of the method).  Some hosts cannot
+ * allocate on the library's behalf: an engine or plugin interface that owns
+ * every device allocation and passes no workspace pointer, or a caller that
+ * must avoid cudaMalloc because it may synchronise the device and fragment a
+ * memory pool the engine manages.  This call takes its scratch (block maxima
+ * and chosen block ids) from a fixed 16 MiB array that the library keeps in
+ * device memory; every GPU that loads the library holds that array until the
+ * process exits.  It allocates nothing.
+ *   - Arguments, outputs and results are those of hs2_block_select.
+ *   - Limit: the scratch hs2_block_select_workspace_size reports for the same
+ *     arguments must be at most 16 MiB (16,777,216 bytes); larger problems
+ *     return HS2_ERR_WORKSPACE and launch nothing.
+ *   - The first call on a device looks up the array's device address (a CUDA
+ *     runtime query, no allocation); make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents.  Nothing in it needs to start at zero: every entry a call reads
+ *     was written earlier in the same call.  Calls that overlap on the GPU
+ *     (different streams, or host threads without ordering) race on it:
+ *     serialise them.
+ */
+hs2_status hs2_block_select_noalloc(const hs2_problem* p, const float* scores,
+                                    int64_t score_stride, int32_t n_blocks, int32_t block,
+                                    int32_t window, int32_t* idx, int32_t* count, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Device error word.  Synchronises ``stream``, returns the first error any

@@ -497,6 +497,54 @@ hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K,
   return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Block selection without a caller workspace.  Some callers cannot hand the
+// library device memory: a host engine or plugin interface that owns every
+// allocation and offers no workspace pointer, or code that must not call
+// cudaMalloc because it can synchronise the device and fragment a memory pool
+// that the engine manages.  For them the scratch of block selection (block
+// maxima and chosen block ids) lives in this fixed array instead.  Every GPU
+// that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace hs2 {
+namespace {
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device.  Host code only
+// sees a stand-in for the array's name, so the address is looked up once per
+// device, with that device current.
+hs2_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HS2_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HS2_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HS2_OK;
+}
+}  // namespace
+}  // namespace hs2
+
+hs2_status hs2_block_select_noalloc(const hs2_problem* p, const float* scores, int64_t score_stride,
+                                    int32_t n_blocks, int32_t block, int32_t window, int32_t* idx,
+                                    int32_t* count, void* stream) {
+  size_t need = 0;
+  hs2_status s = hs2_block_select_workspace_size(p, n_blocks, block, window, &need);
+  if (s != HS2_OK) return s;
+  if (need > kNoAllocScratchBytes) return HS2_ERR_WORKSPACE;  // larger than the fixed scratch
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != HS2_OK) return s;
+  return hs2_block_select(p, scores, score_stride, n_blocks, block, window, idx, count, scratch,
+                          kNoAllocScratchBytes, stream);
+}
+
 hs2_status hs2_get_last_device_error(void* stream) {
   DeviceInfo* dev;
   hs2_status s = device_info(&dev);

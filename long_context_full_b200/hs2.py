@@ -31,7 +31,7 @@ HS2_BF16 = 1
 EXPORTED = [
     "hs2_full_attn_workspace_size", "hs2_full_attn_scores",
     "hs2_topk_workspace_size", "hs2_topk_select",
-    "hs2_block_select_workspace_size", "hs2_block_select",
+    "hs2_block_select_workspace_size", "hs2_block_select", "hs2_block_select_noalloc",
     "hs2_sparse_attn_workspace_size", "hs2_sparse_attn",
     "hs2_get_last_device_error", "hs2_status_string", "hs2_version",
 ]
@@ -77,6 +77,7 @@ def load() -> ctypes.CDLL:
         "hs2_topk_select": [P, vp, i64, i32, i32, vp, vp, vp, sz, vp],
         "hs2_block_select_workspace_size": [P, i32, i32, i32, psz],
         "hs2_block_select": [P, vp, i64, i32, i32, i32, vp, vp, vp, sz, vp],
+        "hs2_block_select_noalloc": [P, vp, i64, i32, i32, i32, vp, vp, vp],
         "hs2_sparse_attn_workspace_size": [P, i32, psz],
         "hs2_sparse_attn": [P, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp],
         "hs2_get_last_device_error": [vp],
@@ -186,6 +187,21 @@ def hs2_block_select(p: Problem, scores, score_stride, n_blocks, block, window, 
     _check(load().hs2_block_select(ctypes.byref(p), _ptr(scores), int(score_stride),
                                    int(n_blocks), int(block), int(window), _ptr(idx),
                                    _ptr(count), w, n, _stream(stream)), "hs2_block_select")
+
+
+# Fixed scratch behind hs2_block_select_noalloc (bytes).
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def hs2_block_select_noalloc(p: Problem, scores, score_stride, n_blocks, block, window, idx,
+                             count, stream=None):
+    """hs2_block_select without a workspace, for callers that cannot provide
+    device memory; the library's fixed 16 MiB scratch is shared by all calls
+    on a device, so calls must not overlap on the GPU."""
+    _check(load().hs2_block_select_noalloc(ctypes.byref(p), _ptr(scores), int(score_stride),
+                                           int(n_blocks), int(block), int(window), _ptr(idx),
+                                           _ptr(count), _stream(stream)),
+           "hs2_block_select_noalloc")
 
 
 def hs2_sparse_attn_workspace_size(p: Problem, idx_stride: int) -> int:
