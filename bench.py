@@ -60,6 +60,27 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
+def rank_first_sequence(rank: int, batch: int) -> int:
+    """Weak scaling: rank r owns global sequences [r * batch, (r + 1) * batch)."""
+    return rank * batch
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (device timings are combined by max)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(batch: int, world: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job query tokens per second: every rank's queries over the slowest rank's time."""
+    return batch * world * steps / (elapsed_ms / 1e3)
+
+
 # ---------------------------------------------------------------------------
 # workload accounting
 # ---------------------------------------------------------------------------
@@ -291,7 +312,7 @@ def main():
     hs2.load()
 
     batch, context = args.batch, args.context
-    w = synth.decode_128k(batch=batch, first_seq=rank * batch, context=context)
+    w = synth.decode_128k(batch=batch, first_seq=rank_first_sequence(rank, batch), context=context)
     workload = WORKLOAD if (batch, context) == (BATCH, CONTEXT) else \
         f"decode_b{batch}_{context}_bf16 (profiling case)"
 
@@ -307,13 +328,6 @@ def main():
     def barrier():
         if world > 1:
             dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---- warm-up
     for _ in range(max(3, args.warmup)):
@@ -348,9 +362,9 @@ def main():
     ph = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
                    for e in ev])
     assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
-    elapsed_ms = max_over_ranks(elapsed_ms)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, "cuda")
     ms_step = elapsed_ms / Kst
-    value = batch * world * Kst / (elapsed_ms / 1e3)
+    value = job_throughput(batch, world, Kst, elapsed_ms)
 
     ab = algorithmic_bytes(batch, context)
     t_full = float(ph[:, 0].mean())
@@ -386,8 +400,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = batch * world * E / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+    e2e_value = job_throughput(batch, world, E, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
