@@ -52,6 +52,10 @@ def parse():
                     help="sequences per GPU (smaller only for profiling captures)")
     ap.add_argument("--context", type=int, default=CONTEXT,
                     help="cached tokens per sequence (smaller only for profiling captures)")
+    ap.add_argument("--workload", default="decode_b8_128k",
+                    choices=["decode_b8_128k", "needle_1m", "ragged_16", "chunk_256k"],
+                    help="other shapes of the pages' workloads (one GPU); the default is the "
+                         "benchmark line")
     return ap.parse_args()
 
 
@@ -84,21 +88,23 @@ def job_throughput(batch: int, world: int, steps: int, elapsed_ms: float) -> flo
 # ---------------------------------------------------------------------------
 # workload accounting
 # ---------------------------------------------------------------------------
-def algorithmic_bytes(batch=BATCH, context=CONTEXT, count=TOPK + WINDOW):
-    """Bytes the step must move at least once (bf16 cache, fp32 scores).
-
-    full attention: K and V read once, Q read, O written, scores written;
-    selection: scores read once; each sparse layer: the selected K/V rows
-    gathered once, its Q read and O written."""
-    kv = 2 * batch * context * HKV * D * 2
-    q = batch * HQ * D * 2
-    scores = batch * HKV * context * 4
-    gather = batch * HKV * count * D * 2 * 2
+def workload_accounting(w, n_layers: int, count=TOPK + WINDOW):
+    """Algorithmic bytes and flops of one step of a synthetic workload: K/V
+    read once, Q read and O written, every visible score written once and read
+    once by the selection, and the selected rows gathered once per layer."""
+    e = 2 if w.dtype == "bf16" else 4
+    tpos = w.query_positions()
+    visible = int((tpos + 1).sum())
+    rows_sel = int(np.minimum(tpos + 1, count).sum())  # selected rows per KV group
+    kv = 2 * int(w.kv_lens.sum()) * w.Hkv * w.D * e
+    q = int(w.q_lens.sum()) * w.Hq * w.D * e
+    scores = visible * w.Hkv * 4
     full = kv + 2 * q + scores
-    select = scores + batch * HKV * (count + 1) * 4
-    sparse = gather + 2 * q
-    return dict(full=full, select=select, sparse_layer=sparse,
-                step=full + select + LAYERS * sparse, kv=kv)
+    select = scores + int(w.q_lens.sum()) * w.Hkv * (count + 1) * 4
+    sparse = rows_sel * w.Hkv * w.D * e * 2 + 2 * q
+    flops = 4 * w.D * w.Hq * visible
+    return dict(full=full, select=select, sparse_layer=sparse, step=full + select + n_layers * sparse,
+                kv=kv, flops=flops, queries=int(w.q_lens.sum()))
 
 
 def peaks():
@@ -109,6 +115,16 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Sustained bf16 tensor throughput (TFLOP/s) for a kernel timed inside a long step."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured sustained"
+    except Exception:
+        return 1400.0, "fallback sustained"
 
 
 def profiled_traffic(kernel_src_hash: str):
@@ -312,17 +328,27 @@ def main():
     hs2.load()
 
     batch, context = args.batch, args.context
-    w = synth.decode_128k(batch=batch, first_seq=rank_first_sequence(rank, batch), context=context)
-    workload = WORKLOAD if (batch, context) == (BATCH, CONTEXT) else \
-        f"decode_b{batch}_{context}_bf16 (profiling case)"
+    if args.workload == "decode_b8_128k":
+        w = synth.decode_128k(batch=batch, first_seq=rank_first_sequence(rank, batch),
+                              context=context)
+        workload = WORKLOAD if (batch, context) == (BATCH, CONTEXT) else \
+            f"decode_b{batch}_{context}_bf16 (profiling case)"
+    else:
+        if world > 1:
+            raise SystemExit("--workload other than the default runs on one GPU")
+        w = {"needle_1m": synth.needle_1m, "ragged_16": synth.ragged_16,
+             "chunk_256k": synth.chunk_256k}[args.workload]()
+        workload = w.name
+    batch = int(w.q_lens.sum())  # query tokens per step
 
     def dev(a):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
 
     Q, K, V = dev(w.q), dev(w.k), dev(w.v)
     QL = [dev(x) for x in w.q_layers]
-    step = HybridBlockStep(HQ, HKV, D, torch.bfloat16, w.q_lens, w.kv_lens, LAYERS, k=TOPK,
-                           window=WINDOW)
+    step = HybridBlockStep(w.Hq, w.Hkv, w.D, torch.bfloat16, w.q_lens, w.kv_lens, w.n_layers,
+                           k=TOPK, window=WINDOW)
+    n_layers = w.n_layers
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -351,7 +377,7 @@ def main():
         e[1].record(stream)
         step.select_tokens()
         e[2].record(stream)
-        for layer in range(LAYERS):
+        for layer in range(n_layers):
             step.sparse_layer(layer, QL[layer], K, V)
         e[3].record(stream)
     end.record(stream)
@@ -366,13 +392,27 @@ def main():
     ms_step = elapsed_ms / Kst
     value = job_throughput(batch, world, Kst, elapsed_ms)
 
-    ab = algorithmic_bytes(batch, context)
+    ab = workload_accounting(w, n_layers)
     t_full = float(ph[:, 0].mean())
     t_sel = float(ph[:, 1].mean())
     t_sp = float(ph[:, 2].mean())
     hbm, hbm_kind = peaks()
-    achieved = ab["full"] / (t_full * 1e-3) / 1e9
-    traffic = profiled_traffic(kernel_sources_hash())
+    chunk = int(w.q_lens.max()) > 1
+    if chunk:  # dense QK^T / PV: the tensor pipe bounds the full-attention call
+        tf, tf_kind = tensor_peak()
+        achieved = ab["flops"] / (t_full * 1e-3) / 1e12
+        roof = {"kernel": "hs2_full_attn_scores (chunk: attention pass + score pass)",
+                "bound": "tensor", "achieved": achieved, "peak": tf, "unit": "TFLOP/s",
+                "frac": achieved / tf, "peak_kind": tf_kind, "traffic": None,
+                "algorithmic_flops": ab["flops"]}
+    else:
+        achieved = ab["full"] / (t_full * 1e-3) / 1e9
+        traffic = profiled_traffic(kernel_sources_hash()) if workload == WORKLOAD else None
+        roof = {"kernel": "hs2_full_attn_scores (decode pass + combine + score finalize)",
+                "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_kind": hbm_kind,
+                "traffic": traffic, "algorithmic_bytes": ab["full"],
+                "frac_of_8TBps": achieved / 8000.0}
 
     # ---- end to end through the public API with host buffers
     pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -404,7 +444,7 @@ def main():
     e2e_value = job_throughput(batch, world, E, e2e_ms)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "decode_b8_128k":
         cpu = cpu_baseline(w)
 
     if rank == 0:
@@ -413,20 +453,17 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) Q/K/V, Philox streams)",
-            "config": {"workload": workload, "batch_per_gpu": batch, "context": context,
-                       "Hq": HQ, "Hkv": HKV, "D": D, "k": TOPK, "window": WINDOW,
-                       "reuse_layers": LAYERS,
+            "config": {"workload": workload, "query_tokens_per_gpu": batch,
+                       "context": int(w.kv_lens.max()), "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                       "k": TOPK, "window": WINDOW, "reuse_layers": n_layers,
                        "l2": f"inputs larger than L2: {ab['kv'] / 2**30:.2f} GiB of K/V streamed per step",
                        "parallelism": f"dp{world} (independent sequences per GPU)"},
             "kv_scan_gbs": ab["kv"] / (t_full * 1e-3) / 1e9,
             "step_gbs": ab["step"] / (ms_step * 1e-3) / 1e9,
+            "step_frac_of_hbm": ab["step"] / (ms_step * 1e-3) / 1e9 / hbm,
             "phase_ms": {"full_attn_scores": t_full, "topk_select": t_sel,
-                         "sparse_attn_x4": t_sp},
-            "roofline": {"kernel": "hs2_full_attn_scores (decode pass + combine + score finalize)",
-                         "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "peak_kind": hbm_kind,
-                         "traffic": traffic, "algorithmic_bytes": ab["full"],
-                         "frac_of_8TBps": achieved / 8000.0},
+                         f"sparse_attn_x{n_layers}": t_sp},
+            "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E},
             "gpu_launches": Kst * step.launches_per_step(),

@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
 
   // -------------------------------------------------------------- consumers
   const bf16* Q = static_cast<const bf16*>(a.Q);
+  const uint64_t keep = policy_evict_last();
   const int r = lane >> 2, qd = lane & 3;
   const float NEG = -INFINITY;
   int stage = 0;
@@ -183,17 +184,19 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
         const float x0 = vlo ? c[0] * a.scale : NEG, x1 = vlo ? c[1] * a.scale : NEG;
         const float x2 = vhi ? c[2] * a.scale : NEG, x3 = vhi ? c[3] * a.scale : NEG;
         // logits of the real heads
+        // logits are read back by the score finalize right after this pass:
+        // ask L2 to keep them (the K/V stream is loaded evict-first)
         if (h1 < a.G && (a.G & 1) == 0) {  // even G: the pair is 8-byte aligned
-          if (vlo) *reinterpret_cast<float2*>(lg + klo * a.Hq + h0) = make_float2(x0, x1);
-          if (vhi) *reinterpret_cast<float2*>(lg + khi * a.Hq + h0) = make_float2(x2, x3);
+          if (vlo) st_hint_f2(lg + klo * a.Hq + h0, x0, x1, keep);
+          if (vhi) st_hint_f2(lg + khi * a.Hq + h0, x2, x3, keep);
         } else {
           if (h0 < a.G) {
-            if (vlo) lg[klo * a.Hq + h0] = x0;
-            if (vhi) lg[khi * a.Hq + h0] = x2;
+            if (vlo) st_hint_f1(lg + klo * a.Hq + h0, x0, keep);
+            if (vhi) st_hint_f1(lg + khi * a.Hq + h0, x2, keep);
           }
           if (h1 < a.G) {
-            if (vlo) lg[klo * a.Hq + h1] = x1;
-            if (vhi) lg[khi * a.Hq + h1] = x3;
+            if (vlo) st_hint_f1(lg + klo * a.Hq + h1, x1, keep);
+            if (vhi) st_hint_f1(lg + khi * a.Hq + h1, x3, keep);
           }
         }
         // online softmax over the 16 keys of this warp, per head (column)
@@ -438,6 +441,7 @@ __global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_const
   float* fst = fsm + 2 * (size_t)kFinKeys * pitch;  // (m_h, 1 / l_h) of the tile's query
   const bool vec = (Hq & 3) == 0;
   const bool vec4 = vec && (a.G & 3) == 0;
+  const uint64_t dead = policy_evict_first();  // each logit is read once
 
   // issue the copy of one tile into buffer k (all threads)
   auto load_tile = [&](int64_t tile, int k) -> bool {
@@ -450,7 +454,7 @@ __global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_const
       const int per_key = Hq / 4;
       for (int i = threadIdx.x; i < nk * per_key; i += kFinKeys) {
         const int key = i / per_key, c = i % per_key;
-        cp_async16(dst + key * pitch + c * 4, src + (int64_t)key * Hq + c * 4, 16);
+        cp_async16_hint(dst + key * pitch + c * 4, src + (int64_t)key * Hq + c * 4, dead);
       }
     } else {
       for (int i = threadIdx.x; i < nk * Hq; i += kFinKeys) dst[(i / Hq) * pitch + i % Hq] = __ldg(src + i);

@@ -14,6 +14,7 @@
 #include "select.cuh"
 #include "sparse_attn.cuh"
 #include "chunk_attn.cuh"
+#include "chunk_tc.cuh"
 
 namespace hs2 {
 
@@ -39,6 +40,15 @@ DeviceInfo g_dev[kMaxDevices];
 size_t finalize_smem(int Hq) { return (2 * (size_t)kFinKeys * (Hq + 4) + 2 * (size_t)Hq) * sizeof(float); }
 std::mutex g_dev_mu;
 
+template <int G>
+cudaError_t set_chunk_tc_smem() {
+  cudaError_t e = cudaFuncSetAttribute(k_chunk_tc<false, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)chunk_tc_smem<false>());
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_chunk_tc<true, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)chunk_tc_smem<true>());
+}
+
 hs2_status device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HS2_ERR_CUDA;
@@ -56,10 +66,8 @@ hs2_status device_info(DeviceInfo** out) {
     if (cudaFuncSetAttribute(k_sparse_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSpSmem) != cudaSuccess)
       return HS2_ERR_CUDA;
-    if (cudaFuncSetAttribute(k_chunk_bf16<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kChStages * 2 * kChKBytes + 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(k_chunk_bf16<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kChStages * kChKBytes + 1024) != cudaSuccess)
+    if (set_chunk_tc_smem<1>() != cudaSuccess || set_chunk_tc_smem<2>() != cudaSuccess ||
+        set_chunk_tc_smem<4>() != cudaSuccess || set_chunk_tc_smem<8>() != cudaSuccess)
       return HS2_ERR_CUDA;
     if (cudaFuncSetAttribute(k_select_cluster<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSelSmemKeys * 4) != cudaSuccess ||
@@ -147,7 +155,10 @@ DecodePlan plan_decode(const hs2_problem* p, const DeviceInfo& dev, void* ws) {
   return pl;
 }
 
-hs2_status encode_kv_map(CUtensorMap* map, const void* base, const hs2_problem* p) {
+// 3-D bf16 tensor map over a [rows, heads, 128] token-major array, boxes of
+// 64 dims x box_heads x box_rows, 128-byte swizzle.
+hs2_status encode_map3(CUtensorMap* map, const void* base, int64_t rows, int heads, int box_heads,
+                       int box_rows) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     cudaDriverEntryPointQueryResult q;
@@ -158,16 +169,19 @@ hs2_status encode_kv_map(CUtensorMap* map, const void* base, const hs2_problem* 
       return HS2_ERR_CUDA;
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
-  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)p->Hkv,
-                              (cuuint64_t)std::max<int64_t>(p->total_kv, 1)};
-  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)p->Hkv * kD * 2};
-  const cuuint32_t box[3] = {64, 1, (cuuint32_t)kDecTile};
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)heads, (cuuint64_t)std::max<int64_t>(rows, 1)};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)heads * kD * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? HS2_OK : HS2_ERR_CUDA;
+}
+
+hs2_status encode_kv_map(CUtensorMap* map, const void* base, const hs2_problem* p) {
+  return encode_map3(map, base, p->total_kv, p->Hkv, 1, kDecTile);
 }
 
 template <int GP>
@@ -241,6 +255,13 @@ hs2_status check_chunk(const hs2_problem* p) {
   return HS2_OK;
 }
 
+template <int G>
+void launch_chunk_tc(dim3 grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const ChunkArgs& a) {
+  k_chunk_tc<false, G><<<grid, kTcThreads, chunk_tc_smem<false>(), st>>>(mq, mk, mv, a);
+  k_chunk_tc<true, G><<<grid, kTcThreads, chunk_tc_smem<true>(), st>>>(mq, mk, mv, a);
+}
+
 template <int GP>
 void launch_chunk_f32(const hs2_problem* p, cudaStream_t st, const ChunkArgs& a) {
   k_chunk_fwd_f32<GP><<<dim3((unsigned)p->total_q, p->Hkv), 128, 0, st>>>(a);
@@ -259,13 +280,19 @@ hs2_status run_chunk(const hs2_problem* p, const DeviceInfo& dev, const void* Q,
   a.total_q = p->total_q; a.total_kv = p->total_kv; a.scale = p->scale;
   a.O = O; a.ml = pl.ml; a.scores = scores; a.stride = stride; a.err = dev.err;
   if (p->dtype == HS2_BF16) {
-    a.QT = kChRows / a.G;
-    CUtensorMap mk, mv;
-    if (encode_kv_map(&mk, K, p) != HS2_OK || encode_kv_map(&mv, V, p) != HS2_OK) return HS2_ERR_CUDA;
+    a.QT = kTcRows / a.G;
+    CUtensorMap mq, mk, mv;
+    if (encode_map3(&mq, Q, p->total_q, p->Hq, a.G, a.QT) != HS2_OK ||
+        encode_map3(&mk, K, p->total_kv, p->Hkv, 1, kTcKeys) != HS2_OK ||
+        encode_map3(&mv, V, p->total_kv, p->Hkv, 1, kTcKeys) != HS2_OK)
+      return HS2_ERR_CUDA;
     const dim3 grid((unsigned)((p->max_q_len + a.QT - 1) / a.QT), p->Hkv, p->B);
-    k_chunk_bf16<false><<<grid, 32 * (kChWarps + 1), kChStages * 2 * kChKBytes + 1024, st>>>(mk, mv, a);
-    if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    k_chunk_bf16<true><<<grid, 32 * (kChWarps + 1), kChStages * kChKBytes + 1024, st>>>(mk, mv, a);
+    switch (a.G) {
+      case 1: launch_chunk_tc<1>(grid, st, mq, mk, mv, a); break;
+      case 2: launch_chunk_tc<2>(grid, st, mq, mk, mv, a); break;
+      case 4: launch_chunk_tc<4>(grid, st, mq, mk, mv, a); break;
+      default: launch_chunk_tc<8>(grid, st, mq, mk, mv, a); break;
+    }
     return launch_status();
   }
   a.QT = 1;

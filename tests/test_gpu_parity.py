@@ -223,7 +223,7 @@ def test_chunk_causal(dtype):
 
 
 def test_chunk_gqa_bf16():
-    for Hq, Hkv in ((4, 4), (8, 2), (32, 4)):
+    for Hq, Hkv in ((4, 4), (8, 4), (8, 2), (32, 4)):
         w = synth.make_workload("chunkg", 62, "bf16", Hq, Hkv, 128, [2500], [150], 1)
         full_check(w)
 
