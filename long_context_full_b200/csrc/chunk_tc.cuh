@@ -23,6 +23,8 @@
 // buffer at columns 0-255, O at 256-383, P (bf16) double buffer at 384-511.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "ptx.cuh"
 #include "chunk_attn.cuh"
@@ -187,17 +189,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     const int64_t hrow = (c.q0 + qr) * a.Hq + (int64_t)g * G + hr;
     const int64_t t_min = c.t0;  // every row sees at least keys [0, t0]
-    // Softmax in base 2: x = s * scale * log2(e), so exp(s*scale - m) = 2^(x - m2)
-    // with m2 = m * log2(e); the row statistics (m2, l) are kept in that form.
+    // Softmax in base 2: with c2 = scale * log2(e), exp(scale*s - m) = 2^(c2*s - m2)
+    // where m2 = m * log2(e); the row statistics (m2, l) are kept in that form.
+    // Pass B folds the normalisation into the exponent: P = 2^(c2*s - (m2 + log2 l)).
     const float c2 = a.scale * 1.4426950408889634f;
-    float m = -INFINITY, l = 0.f, il = 0.f;
-    if (OUT) {
-      m = rv ? a.ml[hrow * 2] : 0.f;  // rows past the chunk: P = 0 rather than NaN
-      l = rv ? a.ml[hrow * 2 + 1] : 0.f;
-      il = l > 0.f ? 1.f / l : 0.f;
+    float m = -INFINITY, l = 0.f, mb = 0.f;
+    if (OUT && rv) {
+      m = a.ml[hrow * 2];
+      l = a.ml[hrow * 2 + 1];
+      mb = m + log2f(l);  // l >= 1: the row's largest logit contributes 1
     }
     float* srow = a.scores + ((c.q0 + qr) * a.Hkv + g) * a.stride;
     const bool v4 = ((reinterpret_cast<uintptr_t>(a.scores) | ((uintptr_t)a.stride * 4)) & 15) == 0;
+    // Every tcgen05.ld/st and full-mask shuffle below must be reached by the
+    // whole warp: the branches around them use warp-uniform conditions only.
+    const bool all_rv = __all_sync(0xffffffffu, rv);
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
@@ -205,44 +211,63 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         record_error(a.err, HS2_ERR_TIMEOUT);
         ok = false;
       }
+      ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok) {
+        // this warp's 64 keys of the tile: k0 .. k0+63
         const int64_t k0 = (int64_t)j * kTcKeys + half * 64;
         uint32_t r[2][32];
         tmem_ld32(trow + b * kTcKeys + half * 64, r[0]);
         tmem_ld32(trow + b * kTcKeys + half * 64 + 32, r[1]);
         tmem_wait_ld();
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int64_t kc = k0 + cc * 32;
-          const bool full = rv && kc + 31 <= t_min;  // no key of the chunk is masked for any row
-          float x[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            x[i] = (full || (rv && kc + i <= t)) ? __uint_as_float(r[cc][i]) * c2 : -INFINITY;
+        auto S = [&](int i) { return __uint_as_float(r[i >> 5][i & 31]); };
+        // MASKED: some key of the 64 lies past some row's position (or rows past the chunk)
+        auto body = [&](auto masked_c) {
+          constexpr bool MASKED = decltype(masked_c)::value;
+          // keys k0 .. k0+nv-1 are visible to this row
+          const int nv = MASKED ? (rv ? (int)max((int64_t)0, min((int64_t)64, t - k0 + 1)) : 0) : 64;
+          auto valid = [nv](int i) { return !MASKED || i < nv; };
           if (!OUT) {
-            float cm = x[0];
+            float mx[8];
 #pragma unroll
-            for (int i = 1; i < 32; ++i) cm = fmaxf(cm, x[i]);
-            const float mn = fmaxf(m, cm);
-            if (mn != -INFINITY) {
-              float sum = 0.f;
+            for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) sum += ex2_approx(x[i] - mn);
-              l = l * ex2_approx(m - mn) + sum;
+            for (int i = 0; i < 64; ++i)
+              mx[i & 7] = fmaxf(mx[i & 7], valid(i) ? S(i) : -INFINITY);
+            const float cm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            if (cm != -INFINITY) {
+              const float mn = fmaxf(m, cm * c2);
+              float sm[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) sm[u] = 0.f;
+#pragma unroll
+              for (int i = 0; i < 64; ++i) {
+                const float e = ex2_approx(fmaf(S(i), c2, -mn));
+                sm[i & 7] += valid(i) ? e : 0.f;
+              }
+              l = l * ex2_approx(m - mn) +
+                  (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
               m = mn;
             }
           } else {
-            float p[32];
+            float p[64];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) p[i] = ex2_approx(x[i] - m) * il;
-            // P (bf16): 32 keys -> 16 packed columns of this tile's P buffer
-            uint32_t pk[16];
+            for (int i = 0; i < 64; ++i) {
+              const float e = ex2_approx(fmaf(S(i), c2, -mb));
+              p[i] = valid(i) ? e : 0.f;
+            }
+            // P (bf16) into this tile's P buffer: 64 keys -> 32 packed columns
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(p[2 * i], p[2 * i + 1]);
-            tmem_st16(trow + kColP + b * (kTcKeys / 2) + (half * 2 + cc) * 16, pk);
-            // scores: sum over the G rows of this query (consecutive lanes) by a
-            // reduce-scatter butterfly; each lane ends with 32/G consecutive keys
+            for (int cc = 0; cc < 2; ++cc) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(p[32 * cc + 2 * i], p[32 * cc + 2 * i + 1]);
+              tmem_st16(trow + kColP + b * (kTcKeys / 2) + half * 32 + cc * 16, pk);
+            }
+            // scores: sum over the G rows of each query (consecutive lanes) by a
+            // reduce-scatter butterfly on both 32-key chunks; each lane ends with
+            // 32/G consecutive keys of each chunk, at offset ``off``
             int off = 0, n = 32;
 #pragma unroll
             for (int msk = G / 2; msk >= 1; msk >>= 1) {
@@ -250,28 +275,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               n >>= 1;
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                if (i < n) {
-                  const float send = up ? p[i] : p[i + n];
-                  const float keep = up ? p[i + n] : p[i];
-                  p[i] = keep + __shfl_xor_sync(0xffffffffu, send, msk);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                  if (i < n) {
+                    float* q = p + 32 * cc;
+                    const float send = up ? q[i] : q[i + n];
+                    const float keep = up ? q[i + n] : q[i];
+                    q[i] = keep + __shfl_xor_sync(0xffffffffu, send, msk);
+                  }
                 }
               }
               if (up) off += n;
             }
-            if (full && v4) {
-              float4* dst = reinterpret_cast<float4*>(srow + kc + off);
 #pragma unroll
-              for (int i = 0; i < 32 / G / 4; ++i)
-                dst[i] = make_float4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-            } else if (rv) {
+            for (int cc = 0; cc < 2; ++cc) {
+              const int64_t kc = k0 + 32 * cc + off;
+              if (!MASKED && v4) {
+                float4* dst = reinterpret_cast<float4*>(srow + kc);
 #pragma unroll
-              for (int i = 0; i < 32 / G; ++i) {
-                const int64_t key = kc + off + i;
-                if (key <= t) srow[key] = p[i];
+                for (int i = 0; i < 32 / G / 4; ++i)
+                  dst[i] = make_float4(p[32 * cc + 4 * i], p[32 * cc + 4 * i + 1],
+                                       p[32 * cc + 4 * i + 2], p[32 * cc + 4 * i + 3]);
+              } else if (rv) {
+#pragma unroll
+                for (int i = 0; i < 32 / G; ++i)
+                  if (kc + i <= t) srow[kc + i] = p[32 * cc + i];
               }
             }
           }
-        }
+        };
+        if (all_rv && k0 + 63 <= t_min) body(std::false_type{});
+        else body(std::true_type{});
       }
       if (OUT) tmem_wait_st();
       tc_fence_before();
@@ -297,6 +331,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         record_error(a.err, HS2_ERR_TIMEOUT);
         ok = false;
       }
+      ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       bf16* O = static_cast<bf16*>(a.O);
 #pragma unroll 1
