@@ -74,7 +74,17 @@ hs2_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(k_select_cluster<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSelSmemKeys * 4) != cudaSuccess)
       return HS2_ERR_CUDA;
+    constexpr int ss_smem = kSsCap * 8 + kSsSortMax * 4;
+    if (cudaFuncSetAttribute(k_select_sampled<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ss_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(k_select_sampled<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ss_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(k_select_sampled<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ss_smem) != cudaSuccess)
+      return HS2_ERR_CUDA;
     d.cluster16 = cudaFuncSetAttribute(k_select_cluster<16>,
+                                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+                  cudaFuncSetAttribute(k_select_sampled<16>,
                                        cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
     cudaGetLastError();  // a refused non-portable size is not an error
     if (cudaFuncSetAttribute(k_finalize_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -322,16 +332,20 @@ hs2_status run_select(const hs2_problem* p, const DeviceInfo& dev, const float* 
   a.B = p->B; a.Hkv = p->Hkv; a.rows = rows; a.k = k; a.window = window; a.block = block;
   a.out = out; a.out_stride = out_stride; a.err = dev.err;
   const int64_t len = std::max<int64_t>(1, max_len);
-  const int cs = (dev.cluster16 && len > 8 * (int64_t)kSelSmemKeys) ? 16 : 8;
+  // k <= kSsSortMax: the sample-guided kernel, one CTA per row when the rows
+  // alone fill the GPU, else a cluster per row; larger k: the exact kernel
+  const bool sampled = k <= kSsSortMax;
+  int cs = (dev.cluster16 && len > 8 * (int64_t)kSelSmemKeys) ? 16 : 8;
+  if (sampled && rows >= 2 * (int64_t)dev.sms) cs = 1;
   int64_t S = (len + cs - 1) / cs;
   S = (S + kSelChunkAlign - 1) / kSelChunkAlign * kSelChunkAlign;
   a.slice = S;
-  a.smem_keys = S <= kSelSmemKeys ? 1 : 0;
+  a.smem_keys = (!sampled && S <= kSelSmemKeys) ? 1 : 0;
   if (rows * cs >= (int64_t(1) << 31)) return HS2_ERR_UNSUPPORTED;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * cs));
   cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = a.smem_keys ? (size_t)S * 4 : 0;
+  cfg.dynamicSmemBytes = sampled ? (size_t)kSsCap * 8 + kSsSortMax * 4 : (a.smem_keys ? (size_t)S * 4 : 0);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -340,8 +354,14 @@ hs2_status run_select(const hs2_problem* p, const DeviceInfo& dev, const float* 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cs == 16 ? cudaLaunchKernelEx(&cfg, k_select_cluster<16>, a, count)
-                                  : cudaLaunchKernelEx(&cfg, k_select_cluster<8>, a, count);
+  cudaError_t e;
+  if (sampled)
+    e = cs == 16 ? cudaLaunchKernelEx(&cfg, k_select_sampled<16>, a, count)
+                 : (cs == 8 ? cudaLaunchKernelEx(&cfg, k_select_sampled<8>, a, count)
+                            : cudaLaunchKernelEx(&cfg, k_select_sampled<1>, a, count));
+  else
+    e = cs == 16 ? cudaLaunchKernelEx(&cfg, k_select_cluster<16>, a, count)
+                 : cudaLaunchKernelEx(&cfg, k_select_cluster<8>, a, count);
   return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 

@@ -181,6 +181,45 @@ def test_select_rows_longer_than_shared_memory():
         assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
 
 
+def test_select_many_long_rows():
+    """Enough rows to fill the GPU with one CTA per row, rows longer than a
+    CTA's candidate buffer: the sampled threshold, then the exact select."""
+    rng = np.random.default_rng(31)
+    R, n = 320, 30000
+    S = rng.standard_normal((R, n)).astype(np.float32)
+    S[: R // 2, -5000:] += np.float32(2.0)  # top keys crowded at the end for half the rows
+    ts = [n - 1 - 11 * r for r in range(R)]
+    idx, cnt = gpu_select_on(S, ts)
+    for r in range(0, R, 5):
+        oi, oc = oracle.topk_select(S[r], ts[r])
+        assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
+
+
+@pytest.mark.parametrize("R,n", [(300, 20000), (2, 50000), (2, 600000)])
+def test_select_all_equal_falls_back_to_exact(R, n):
+    """Every key ties: more keys reach the sampled threshold than a CTA holds,
+    so the exact selection over global memory runs (one CTA per row, and a
+    16-CTA cluster per row)."""
+    S = np.full((R, n), np.float32(0.5))
+    ts = [n - 1 - 3 * r for r in range(R)]
+    idx, cnt = gpu_select_on(S, ts)
+    for r in range(0, R, max(1, R // 20)):
+        oi, oc = oracle.topk_select(S[r], ts[r])
+        assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
+
+
+def test_select_large_k_exact_kernel():
+    """k above the sampled kernel's limit runs the exact cluster kernel."""
+    rng = np.random.default_rng(37)
+    n = 50000
+    S = rng.integers(0, 500, (3, n)).astype(np.float32)
+    ts = [n - 1, 30000, 2500]
+    idx, cnt = gpu_select_on(S, ts, k=3000)
+    for r in range(3):
+        oi, oc = oracle.topk_select(S[r], ts[r], 3000, 128)
+        assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
+
+
 @pytest.mark.parametrize("stride_extra", [1, 2, 3, 37])
 def test_select_unaligned_stride(stride_extra):
     """Score rows whose stride is not a multiple of 4 floats (the C ABI allows
