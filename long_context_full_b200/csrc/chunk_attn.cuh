@@ -67,6 +67,7 @@ __device__ __forceinline__ bool chunk_tile(const ChunkArgs& a, ChTile& c) {
 // ----------------------------------------------------------------------------
 template <int GP>
 __global__ void __launch_bounds__(128) k_chunk_fwd_f32(const __grid_constant__ ChunkArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   const int64_t qi = blockIdx.x;
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(128) k_chunk_fwd_f32(const __grid_constant__ C
 // 8w..8w+7 of the block: recomputed logits, normalised, summed over the group.
 template <int GP>
 __global__ void __launch_bounds__(128) k_chunk_scores_f32(const __grid_constant__ ChunkArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   const int64_t qi = blockIdx.z;
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

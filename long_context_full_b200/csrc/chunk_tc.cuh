@@ -48,6 +48,7 @@ template <bool OUT, int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_chunk_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ ChunkArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   constexpr int kStage = (OUT ? 2 : 1) * kTcTileBytes;
   constexpr uint32_t kCols = OUT ? 512 : 256;  // S double buffer (+ O and P)
   constexpr uint32_t kColO = 2 * kTcKeys, kColP = 3 * kTcKeys;

@@ -75,6 +75,7 @@ template <int NST>
 __global__ void __launch_bounds__(32 * (kDecWarps + 1))
     k_decode_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ DecodeArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full_bar[NST];
   __shared__ __align__(8) uint64_t empty_bar[NST];
@@ -271,6 +272,7 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
 // ----------------------------------------------------------------------------
 template <int GP>
 __global__ void __launch_bounds__(32 * kDecWarps) k_decode_f32(const __grid_constant__ DecodeArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.x, g = blockIdx.y;
   const float* Q = static_cast<const float*>(a.Q);
@@ -333,6 +335,7 @@ constexpr int kCombStage = 64;  // partial rows staged in shared memory per roun
 template <typename OT>
 __global__ void __launch_bounds__(kD) k_decode_combine(const __grid_constant__ DecodeArgs a, OT* O,
                                                        float* ml) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   const int b = blockIdx.x, g = blockIdx.y, hl = blockIdx.z, d = threadIdx.x;
   if (b == 0 && g == 0 && hl == 0 && d == 0) {
     if (__ldg(a.kvoff + a.B) != a.total_kv || __ldg(a.qoff + a.B) != a.total_q)
@@ -434,6 +437,7 @@ __device__ __forceinline__ bool fin_tile(const DecodeArgs& a, int64_t tile, int 
 __global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_constant__ DecodeArgs a,
                                                               const float* ml, float* scores,
                                                               int64_t stride, int ntile_seq) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ __align__(16) float fsm[];  // 2 x [kFinKeys][Hq + 4] logits, [Hq][2] stats
   const int Hq = a.Hq, pitch = Hq + 4;
   const int64_t ntiles = (int64_t)a.B * ntile_seq;

@@ -22,6 +22,35 @@ __device__ int g_device_error;  // first error recorded by a kernel, 0 if none
 
 namespace {
 
+// Launches ``kern`` on ``st`` with programmatic dependent launch allowed (each
+// kernel starts with griddepcontrol.wait, so nothing is read or written before
+// the previous kernel on the stream has finished) and, if cluster > 0, in
+// thread-block clusters of that many CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = (unsigned)n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 constexpr int kMaxDevices = 64;
 constexpr int kDecStages = 3;     // bf16 decode ring depth (2 CTAs per SM)
 constexpr int kMaxHq = 192;      // query heads the score finalize can stage
@@ -196,7 +225,7 @@ hs2_status encode_kv_map(CUtensorMap* map, const void* base, const hs2_problem* 
 
 template <int GP>
 void launch_decode_f32(dim3 grid, cudaStream_t st, const DecodeArgs& a) {
-  k_decode_f32<GP><<<grid, 32 * kDecWarps, 0, st>>>(a);
+  launch(k_decode_f32<GP>, dim3(grid), dim3(32 * kDecWarps), 0, st, 0, a);
 }
 
 hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q, const void* K,
@@ -213,9 +242,9 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
   if (p->dtype == HS2_BF16) {
     CUtensorMap mk, mv;
     if (encode_kv_map(&mk, K, p) != HS2_OK || encode_kv_map(&mv, V, p) != HS2_OK) return HS2_ERR_CUDA;
-    k_decode_bf16<kDecStages><<<grid, 32 * (kDecWarps + 1), kDecStages * kDecStageBytes + 1024, st>>>(mk, mv, a);
+    launch(k_decode_bf16<kDecStages>, dim3(grid), dim3(32 * (kDecWarps + 1)), kDecStages * kDecStageBytes + 1024, st, 0, mk, mv, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    k_decode_combine<bf16><<<dim3(p->B, p->Hkv, a.G), kD, 0, st>>>(a, static_cast<bf16*>(O), pl.ml);
+    launch(k_decode_combine<bf16>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<bf16*>(O), pl.ml);
   } else {
     const int G = a.G;
     if (G <= 1) launch_decode_f32<1>(grid, st, a);
@@ -224,7 +253,7 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     else if (G <= 8) launch_decode_f32<8>(grid, st, a);
     else launch_decode_f32<16>(grid, st, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    k_decode_combine<float><<<dim3(p->B, p->Hkv, a.G), kD, 0, st>>>(a, static_cast<float*>(O), pl.ml);
+    launch(k_decode_combine<float>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<float*>(O), pl.ml);
   }
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
   if (p->max_kv_len > 0) {
@@ -233,7 +262,7 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     int per_sm = 1;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_finalize_scores, kFinKeys, finalize_smem(p->Hq));
     const int64_t grid = std::min<int64_t>(ntiles, (int64_t)std::max(1, per_sm) * dev.sms);
-    k_finalize_scores<<<(unsigned)grid, kFinKeys, finalize_smem(p->Hq), st>>>(a, pl.ml, scores, stride,
+    launch(k_finalize_scores, dim3((unsigned)grid), dim3(kFinKeys), finalize_smem(p->Hq), st, 0, a, pl.ml, scores, stride,
                                                                                ntile_seq);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
   }
@@ -268,14 +297,14 @@ hs2_status check_chunk(const hs2_problem* p) {
 template <int G>
 void launch_chunk_tc(dim3 grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
                      const CUtensorMap& mv, const ChunkArgs& a) {
-  k_chunk_tc<false, G><<<grid, kTcThreads, chunk_tc_smem<false>(), st>>>(mq, mk, mv, a);
-  k_chunk_tc<true, G><<<grid, kTcThreads, chunk_tc_smem<true>(), st>>>(mq, mk, mv, a);
+  launch(k_chunk_tc<false, G>, dim3(grid), dim3(kTcThreads), chunk_tc_smem<false>(), st, 0, mq, mk, mv, a);
+  launch(k_chunk_tc<true, G>, dim3(grid), dim3(kTcThreads), chunk_tc_smem<true>(), st, 0, mq, mk, mv, a);
 }
 
 template <int GP>
 void launch_chunk_f32(const hs2_problem* p, cudaStream_t st, const ChunkArgs& a) {
-  k_chunk_fwd_f32<GP><<<dim3((unsigned)p->total_q, p->Hkv), 128, 0, st>>>(a);
-  k_chunk_scores_f32<GP><<<dim3((unsigned)((p->max_kv_len + 31) / 32), p->Hkv, (unsigned)p->total_q), 128, 0, st>>>(a);
+  launch(k_chunk_fwd_f32<GP>, dim3(dim3((unsigned)p->total_q, p->Hkv)), dim3(128), 0, st, 0, a);
+  launch(k_chunk_scores_f32<GP>, dim3(dim3((unsigned)((p->max_kv_len + 31) / 32), p->Hkv, (unsigned)p->total_q)), dim3(128), 0, st, 0, a);
 }
 
 hs2_status run_chunk(const hs2_problem* p, const DeviceInfo& dev, const void* Q, const void* K,
@@ -342,26 +371,16 @@ hs2_status run_select(const hs2_problem* p, const DeviceInfo& dev, const float* 
   a.slice = S;
   a.smem_keys = (!sampled && S <= kSelSmemKeys) ? 1 : 0;
   if (rows * cs >= (int64_t(1) << 31)) return HS2_ERR_UNSUPPORTED;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(rows * cs));
-  cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = sampled ? (size_t)kSsCap * 8 + kSsSortMax * 4 : (a.smem_keys ? (size_t)S * 4 : 0);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  const dim3 grid((unsigned)(rows * cs)), threads(kSelThreads);
+  const size_t smem = sampled ? (size_t)kSsCap * 8 + kSsSortMax * 4 : (a.smem_keys ? (size_t)S * 4 : 0);
   cudaError_t e;
   if (sampled)
-    e = cs == 16 ? cudaLaunchKernelEx(&cfg, k_select_sampled<16>, a, count)
-                 : (cs == 8 ? cudaLaunchKernelEx(&cfg, k_select_sampled<8>, a, count)
-                            : cudaLaunchKernelEx(&cfg, k_select_sampled<1>, a, count));
+    e = cs == 16 ? launch(k_select_sampled<16>, grid, threads, smem, st, cs, a, count)
+                 : (cs == 8 ? launch(k_select_sampled<8>, grid, threads, smem, st, cs, a, count)
+                            : launch(k_select_sampled<1>, grid, threads, smem, st, cs, a, count));
   else
-    e = cs == 16 ? cudaLaunchKernelEx(&cfg, k_select_cluster<16>, a, count)
-                 : cudaLaunchKernelEx(&cfg, k_select_cluster<8>, a, count);
+    e = cs == 16 ? launch(k_select_cluster<16>, grid, threads, smem, st, cs, a, count)
+                 : launch(k_select_cluster<8>, grid, threads, smem, st, cs, a, count);
   return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 
@@ -371,19 +390,7 @@ hs2_status run_select(const hs2_problem* p, const DeviceInfo& dev, const float* 
 template <typename Kern>
 cudaError_t launch_cluster(Kern kern, unsigned ctas, unsigned threads, size_t smem, int cs,
                            cudaStream_t st, const SparseArgs& a) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ctas);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  return launch(kern, dim3(ctas), dim3(threads), smem, st, cs, a);
 }
 
 hs2_status check_ws(void* ws, size_t have, size_t need) {
@@ -489,12 +496,12 @@ hs2_status hs2_block_select(const hs2_problem* p, const float* scores, int64_t s
   Carve w(workspace);
   float* bmax = w.take<float>((size_t)rows * nb);
   int32_t* bsel = w.take<int32_t>((size_t)rows * n_blocks);
-  k_block_max<<<dim3((unsigned)rows, (unsigned)((nb + 7) / 8)), 256, 0, st>>>(
+  launch(k_block_max, dim3(dim3((unsigned)rows, (unsigned)((nb + 7) / 8))), dim3(256), 0, st, 0, 
       scores, score_stride, p->q_offsets, p->kv_offsets, p->B, p->Hkv, block, window, bmax, nb, dev->err);
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
   if ((s = run_select(p, *dev, bmax, nb, nb, n_blocks, window, block, bsel, n_blocks, nullptr, st)) != HS2_OK)
     return s;
-  k_block_expand<<<(unsigned)rows, 256, 0, st>>>(bsel, n_blocks, p->q_offsets, p->kv_offsets, p->B,
+  launch(k_block_expand, dim3((unsigned)rows), dim3(256), 0, st, 0, bsel, n_blocks, p->q_offsets, p->kv_offsets, p->B,
                                                  p->Hkv, block, window, idx,
                                                  (int64_t)n_blocks * block + window, count);
   return launch_status();

@@ -149,6 +149,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 
+// Programmatic dependent launch: every kernel of the library starts with this
+// wait, so it may be launched before its predecessor on the stream has
+// finished (its launch overlaps the predecessor's tail) but reads and writes
+// nothing until the predecessor's grid has completed and its memory is
+// visible.  Without a programmatic predecessor it returns at once.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // 2^x by the special-function unit (ex2.approx, flush-to-zero; 2^-inf = +0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -24,6 +24,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace hs2 {
 
@@ -321,6 +322,7 @@ __device__ void sel_exact(cg::cluster_group& cl, SelState<CS>& st, const SelectA
 template <int CS>
 __global__ void __launch_bounds__(kSelThreads) k_select_cluster(const __grid_constant__ SelectArgs a,
                                                                 int32_t* count) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ uint4 skeys4[];
   uint32_t* skeys = reinterpret_cast<uint32_t*>(skeys4);
   __shared__ SelState<CS> st;
@@ -484,6 +486,7 @@ __device__ __forceinline__ void sel_block_find(const uint32_t* hist, int nb, int
 template <int CS>
 __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_constant__ SelectArgs a,
                                                                 int32_t* count) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ uint4 ss_dyn[];
   uint64_t* cand = reinterpret_cast<uint64_t*>(ss_dyn);            // kept: (position << 32 | key)
   int32_t* sel = reinterpret_cast<int32_t*>(cand + kSsCap);       // selected positions
@@ -780,6 +783,7 @@ __global__ void __launch_bounds__(256) k_block_max(const float* scores, int64_t 
                                                    const int64_t* qoff, const int64_t* kvoff, int B,
                                                    int Hkv, int block, int window, float* bmax,
                                                    int64_t bstride, int* err) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   const int64_t r = blockIdx.x;
   const int lane = threadIdx.x & 31;
   const int64_t bi = (int64_t)blockIdx.y * 8 + (threadIdx.x >> 5);
@@ -804,6 +808,7 @@ __global__ void __launch_bounds__(256) k_block_expand(const int32_t* bsel, int n
                                                       const int64_t* qoff, const int64_t* kvoff, int B,
                                                       int Hkv, int block, int window, int32_t* idx,
                                                       int64_t idx_stride, int32_t* count) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   const int64_t r = blockIdx.x;
   const QueryRow q = query_row(qoff, kvoff, B, r / Hkv);
   int64_t nc = q.t - window + 1;

@@ -144,6 +144,7 @@ __device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_
 // fragment scheme as the decode pass (P^T by one movmatrix transpose).
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_constant__ SparseArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ __align__(128) uint8_t sp_smem[];
   __shared__ float wm[kSpWarps * 8], wl[kSpWarps * 8];
   __shared__ float wo[kSpWarps * 8 * kD];
@@ -274,6 +275,7 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
 // ----------------------------------------------------------------------------
 template <int GP>
 __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_f32(const __grid_constant__ SparseArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
   __shared__ float wm[kSpWarps * GP], wl[kSpWarps * GP];
   __shared__ float wo[kSpWarps * GP * kD];
   __shared__ SpRecv recv;
