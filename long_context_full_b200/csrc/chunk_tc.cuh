@@ -8,19 +8,25 @@
 // builds the cache and judges token importance) and "Two-Level KV Sharing: ..."
 // (prefill is dominated by large matrix products).
 //
-// A CTA owns 128 (query, head) rows: 128/G query tokens x the G query heads of
-// one KV group, which share every K/V tile.  Two passes over the visible keys:
-//   pass A (STATS): S = Q K^T per 128-key tile into tensor memory; the softmax
-//                   warps keep each row's running max m and sum l.
-//   pass B (OUT):   S = Q K^T again; P = exp(S - m) / l is exact (no online
-//                   rescaling of O is ever needed); the selection scores (sum of
-//                   P over the G heads of each query) are written; P goes back
-//                   into tensor memory as bf16 and O += P V runs with A read
-//                   from tensor memory.  O is final when the last tile is done.
-// Roles: warps 0-7 softmax (warp w reads tensor-memory lanes 32(w%4).. + 31,
-// one row per thread, and columns 64(w/4)..+63 of each tile), warp 8 TMA
-// producer, warp 9 issues the MMAs (one thread).  Tensor memory: S double
-// buffer at columns 0-255, O at 256-383, P (bf16) double buffer at 384-511.
+// A CTA owns two Q tiles of 128 (query, head) rows each: 128/G query tokens x
+// the G query heads of one KV group per tile, 256/G consecutive queries in all.
+// Every K/V tile it loads feeds both Q tiles.  One kernel, two passes over the
+// visible keys:
+//   pass A: S_t = Q_t K^T per 128-key tile into tensor memory (four S buffers:
+//           two per Q tile); softmax warpgroup t keeps each row's running max
+//           and sum, in registers.
+//   pass B: S_t = Q_t K^T again; P = exp(S - m) / l is exact, so O never needs
+//           rescaling; the selection scores (sum of P over the G heads of each
+//           query) are written; P goes back into the S columns as bf16 (two
+//           keys per column, written behind the columns already read) and
+//           O_t += P V runs with A read from tensor memory.
+// Roles: warpgroup t (warps 4t .. 4t+3) does the softmax of Q tile t, one row
+// per thread (warp w reads tensor-memory lanes 32(w%4) .. +31); warp 8 issues
+// the TMA loads (Q once; K and V through separate two-stage rings); warp 9
+// issues the MMAs from one thread.  Tensor memory (512 columns): pass A, the S
+// buffers (tile t, buffer b) at 256t + 128b; pass B, S_t/P_t at 128t and O_t
+// at 256 + 128t.  Before S_t of the next key tile overwrites P_t, the MMA
+// thread waits for the commit of the O_t += P_t V that reads it.
 #pragma once
 
 #include <type_traits>
@@ -31,60 +37,65 @@
 
 namespace hs2 {
 
-constexpr int kTcRows = 128;                     // rows per CTA = tensor-memory lanes
-constexpr int kTcKeys = 128;                     // keys per tile
-constexpr int kTcStages = 2;                     // K/V ring depth
+constexpr int kTcRows = 128;                     // rows per Q tile = tensor-memory lanes
+constexpr int kTcQTiles = 2;                     // Q tiles per CTA
+constexpr int kTcKeys = 128;                     // keys per K/V tile
+constexpr int kTcStages = 2;                     // depth of the K ring and of the V ring
 constexpr int kTcTileBytes = kTcKeys * kD * 2;   // a K or V tile: two swizzled [128][64] halves
-constexpr int kTcQBytes = kTcRows * kD * 2;
-constexpr int kTcSoftWarps = 8;   // two warpgroups: column halves of every tile
-constexpr int kTcThreads = 32 * (kTcSoftWarps + 2);
+constexpr int kTcQBytes = kTcRows * kD * 2;      // one Q tile
+constexpr int kTcThreads = 32 * 10;              // 2 softmax warpgroups, TMA warp, MMA warp
 
-template <bool OUT>
 constexpr size_t chunk_tc_smem() {
-  return 1024 + kTcQBytes + (size_t)kTcStages * (OUT ? 2 : 1) * kTcTileBytes;
+  return 1024 + (size_t)kTcQTiles * kTcQBytes + 2 * (size_t)kTcStages * kTcTileBytes;
 }
 
-template <bool OUT, int G>
+template <int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_chunk_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ ChunkArgs a) {
   grid_dep_wait();  // the previous kernel on the stream has finished
-  constexpr int kStage = (OUT ? 2 : 1) * kTcTileBytes;
-  constexpr uint32_t kCols = OUT ? 512 : 256;  // S double buffer (+ O and P)
-  constexpr uint32_t kColO = 2 * kTcKeys, kColP = 3 * kTcKeys;
+  constexpr int QT1 = kTcRows / G;  // queries per Q tile
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t q_full;
-  __shared__ __align__(8) uint64_t kv_full[kTcStages], kv_empty[kTcStages];
-  __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_full[2];
-  __shared__ __align__(8) uint64_t o_full;
+  __shared__ __align__(8) uint64_t k_full[kTcStages], k_empty[kTcStages];
+  __shared__ __align__(8) uint64_t v_full[kTcStages], v_empty[kTcStages];
+  __shared__ __align__(8) uint64_t sa_full[2][2], sa_free[2][2];  // pass A: [Q tile][S buffer]
+  __shared__ __align__(8) uint64_t sb_full[2], pb_full[2], pv_done[2], o_full;  // pass B: [Q tile]
   __shared__ uint32_t tmem_base_sh;
 
   ChTile c;
   if (!chunk_tile(a, c)) return;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
-  uint8_t* sKV = base + kTcQBytes;
+  uint8_t* sK = base + kTcQTiles * kTcQBytes;
+  uint8_t* sV = sK + kTcStages * kTcTileBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
   const int64_t nkeys = c.t0 + c.nq;  // keys [0, t_last] are visible to some row
-  const int ntiles = (int)((nkeys + kTcKeys - 1) / kTcKeys);
+  const int n = (int)((nkeys + kTcKeys - 1) / kTcKeys);
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], OUT ? 1 : kTcSoftWarps);  // PV done (commit) / softmax warps read S
-      mbar_init(&p_full[b], kTcSoftWarps);
+    for (int t = 0; t < 2; ++t) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&sa_full[t][b], 1);
+        mbar_init(&sa_free[t][b], 4);  // the four warps of warpgroup t
+      }
+      mbar_init(&sb_full[t], 1);
+      mbar_init(&pb_full[t], 4);
+      mbar_init(&pv_done[t], 1);
     }
     mbar_init(&o_full, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&tmem_base_sh, kCols);
+    tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -92,149 +103,179 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == kTcSoftWarps) {
+  if (warp == 8) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       bool ok = true;
-      mbar_arrive_expect_tx(&q_full, kTcQBytes);
-      tma_load_3d(sQ, &tmQ, &q_full, 0, g * G, (int)c.q0);
-      tma_load_3d(sQ + kTcQBytes / 2, &tmQ, &q_full, 64, g * G, (int)c.q0);
-      uint32_t issued = 0, last_phase = 0;
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int st = j % kTcStages;
-        const uint32_t ph = (uint32_t)(j / kTcStages) & 1u;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1u)) {
-          record_error(a.err, HS2_ERR_TIMEOUT);
-          ok = false;
-          break;
-        }
-        uint8_t* sk = sKV + st * kStage;
-        const int key = (int)(c.kv0 + (int64_t)j * kTcKeys);
-        mbar_arrive_expect_tx(&kv_full[st], kStage);
-        tma_load_3d(sk, &tmK, &kv_full[st], 0, g, key);
-        tma_load_3d(sk + kTcTileBytes / 2, &tmK, &kv_full[st], 64, g, key);
-        if (OUT) {
-          tma_load_3d(sk + kTcTileBytes, &tmV, &kv_full[st], 0, g, key);
-          tma_load_3d(sk + kTcTileBytes + kTcTileBytes / 2, &tmV, &kv_full[st], 64, g, key);
-        }
-        issued |= 1u << st;
-        last_phase = (last_phase & ~(1u << st)) | (ph << st);
+      mbar_arrive_expect_tx(&q_full, kTcQTiles * kTcQBytes);
+      for (int t = 0; t < kTcQTiles; ++t) {
+        tma_load_3d(sQ + t * kTcQBytes, &tmQ, &q_full, 0, g * G, (int)(c.q0 + t * QT1));
+        tma_load_3d(sQ + t * kTcQBytes + kTcQBytes / 2, &tmQ, &q_full, 64, g * G, (int)(c.q0 + t * QT1));
       }
+      // K fills 0 .. 2n-1 (pass A tiles, then pass B tiles); V fills 0 .. n-1
+      auto fill = [&](uint64_t* full, uint64_t* empty, uint8_t* ring, const CUtensorMap* map, int f,
+                      int j) -> bool {
+        const int st = f % kTcStages;
+        if (!mbar_wait(&empty[st], ((uint32_t)(f / kTcStages) & 1u) ^ 1u)) return false;
+        const int key = (int)(c.kv0 + (int64_t)j * kTcKeys);
+        uint8_t* dst = ring + st * kTcTileBytes;
+        mbar_arrive_expect_tx(&full[st], kTcTileBytes);
+        tma_load_3d(dst, map, &full[st], 0, g, key);
+        tma_load_3d(dst + kTcTileBytes / 2, map, &full[st], 64, g, key);
+        return true;
+      };
+      int kf = 0, vf = 0;
+      for (int j = 0; j < n && ok; ++j) {
+        if ((ok = fill(k_full, k_empty, sK, &tmK, kf, j))) ++kf;
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        if (!(ok = fill(k_full, k_empty, sK, &tmK, kf, j))) break;
+        ++kf;
+        if (!(ok = fill(v_full, v_empty, sV, &tmV, vf, j))) break;
+        ++vf;
+      }
+      if (!ok) record_error(a.err, HS2_ERR_TIMEOUT);
       // before the CTA exits: every fill issued here has landed, and every
       // release of a stage (an MMA commit) has arrived
       if (!mbar_wait(&q_full, 0)) record_error(a.err, HS2_ERR_TIMEOUT);
-      for (int s = 0; s < kTcStages; ++s)
-        if ((issued >> s) & 1u) {
-          if (!mbar_wait(&kv_full[s], (last_phase >> s) & 1u)) record_error(a.err, HS2_ERR_TIMEOUT);
-          if (ok && !mbar_wait(&kv_empty[s], (last_phase >> s) & 1u)) record_error(a.err, HS2_ERR_TIMEOUT);
+      auto drain = [&](uint64_t* full, uint64_t* empty, int nf) {
+        for (int f = nf - kTcStages; f < nf; ++f) {
+          if (f < 0) continue;
+          const uint32_t ph = (uint32_t)(f / kTcStages) & 1u;
+          if (!mbar_wait(&full[f % kTcStages], ph)) record_error(a.err, HS2_ERR_TIMEOUT);
+          if (ok && !mbar_wait(&empty[f % kTcStages], ph)) record_error(a.err, HS2_ERR_TIMEOUT);
         }
+      };
+      drain(k_full, k_empty, kf);
+      drain(v_full, v_empty, vf);
     }
-  } else if (warp == kTcSoftWarps + 1) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(kTcRows, kTcKeys, 0, 0);  // Q K^T: both K-major
       constexpr uint32_t idesc_o = umma_idesc_bf16(kTcRows, kD, 0, 1);       // P V: V is MN-major
       bool ok = mbar_wait(&q_full, 0);
-      if (!ok) record_error(a.err, HS2_ERR_TIMEOUT);
       tc_fence_after();
-      const uint32_t qa = smem_u32(sQ);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kTcStages, b = j & 1;
-        if (!mbar_wait(&kv_full[st], (uint32_t)(j / kTcStages) & 1u)) return false;
-        if (!mbar_wait(&s_free[b], ((uint32_t)(j >> 1) & 1u) ^ 1u)) return false;
-        tc_fence_after();
-        const uint32_t kb = smem_u32(sKV + st * kStage);
+      const uint32_t qa0 = smem_u32(sQ);
+      // S (128 x 128) = Q_t K^T into tensor columns d_col
+      auto mma_s = [&](uint32_t d_col, int t, int kst) {
+        const uint32_t qa = qa0 + t * kTcQBytes;
+        const uint32_t kb = smem_u32(sK + kst * kTcTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kTcTileBytes / 2) + (kk & 3) * 32;
-          umma_ss(tmem + b * kTcKeys, umma_desc_sw128(qa + off, 16, 1024),
-                  umma_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+          umma_ss(tmem + d_col, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
+                  idesc_s, kk > 0);
         }
-        umma_commit(&s_full[b]);
-        if (!OUT) umma_commit(&kv_empty[st]);
-        return true;
       };
-      if (ok && ntiles > 0) ok = issue_s(0);
-      for (int j = 0; j < ntiles && ok; ++j) {
-        if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
-        if (OUT) {
-          const int st = j % kTcStages, b = j & 1;
-          if (!(ok = mbar_wait(&p_full[b], (uint32_t)(j >> 1) & 1u))) break;
+      auto kwait = [&](int f) { return mbar_wait(&k_full[f % kTcStages], (uint32_t)(f / kTcStages) & 1u); };
+      // ---- pass A
+      for (int j = 0; j < n && ok; ++j) {
+        if (!(ok = kwait(j))) break;
+        const int b = j & 1;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!(ok = mbar_wait(&sa_free[t][b], ((uint32_t)(j >> 1) & 1u) ^ 1u))) break;
           tc_fence_after();
-          const uint32_t vb = smem_u32(sKV + st * kStage + kTcTileBytes);
+          mma_s(256 * t + 128 * b, t, j % kTcStages);
+          umma_commit(&sa_full[t][b]);
+        }
+        umma_commit(&k_empty[j % kTcStages]);
+      }
+      // every S buffer of pass A has been read before pass B reuses the columns
+      for (int j = (n > 2 ? n - 2 : 0); j < n && ok; ++j)
+        for (int t = 0; t < 2 && ok; ++t) ok = mbar_wait(&sa_free[t][j & 1], (uint32_t)(j >> 1) & 1u);
+      tc_fence_after();
+      // ---- pass B
+      if (ok && n > 0 && (ok = kwait(n))) {
+        tc_fence_after();
+        mma_s(0, 0, n % kTcStages);
+        umma_commit(&sb_full[0]);
+        mma_s(128, 1, n % kTcStages);
+        umma_commit(&sb_full[1]);
+        umma_commit(&k_empty[n % kTcStages]);
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int vst = j % kTcStages;
+        if (!(ok = mbar_wait(&v_full[vst], (uint32_t)(j / kTcStages) & 1u))) break;
+        const uint32_t vb = smem_u32(sV + vst * kTcTileBytes);
+        const int kf = n + j + 1;  // the K fill of key tile j + 1
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!(ok = mbar_wait(&pb_full[t], (uint32_t)j & 1u))) break;
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTcKeys / 16; ++kk)
-            umma_ts(tmem + kColO, tmem + kColP + b * (kTcKeys / 2) + kk * 8,
+            umma_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8,
                     umma_desc_sw128(vb + kk * 2048, kTcTileBytes / 2, 1024), idesc_o,
                     (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&s_free[b]);
-          umma_commit(&kv_empty[st]);
+          umma_commit(&pv_done[t]);
+          if (t == 1) umma_commit(&v_empty[vst]);
+          if (j + 1 < n) {
+            // P_t is read by the MMAs just issued; S_t of the next tile overwrites it
+            if (!(ok = mbar_wait(&pv_done[t], (uint32_t)j & 1u))) break;
+            if (t == 0 && !(ok = kwait(kf))) break;
+            tc_fence_after();
+            mma_s(128 * t, t, kf % kTcStages);
+            umma_commit(&sb_full[t]);
+            if (t == 1) umma_commit(&k_empty[kf % kTcStages]);
+          }
         }
       }
+      umma_commit(&o_full);
+      // the last commits have arrived before the CTA exits
+      if (ok && n > 0)
+        for (int t = 0; t < 2; ++t)
+          if (!mbar_wait(&pv_done[t], (uint32_t)(n - 1) & 1u)) ok = false;
       if (!ok) record_error(a.err, HS2_ERR_TIMEOUT);
-      if (OUT) {
-        umma_commit(&o_full);
-        // the commits that free the S buffers have arrived before the CTA exits
-        for (int j = (ntiles > 2 ? ntiles - 2 : 0); ok && j < ntiles; ++j)
-          if (!mbar_wait(&s_free[j & 1], (uint32_t)(j >> 1) & 1u)) record_error(a.err, HS2_ERR_TIMEOUT);
-      }
     }
   } else {
-    // --------------------------------------------------------- softmax warps
-    __shared__ float half_ml[2][kTcRows];  // STATS: the upper half's (m, l) per row
-    const int quarter = warp & 3, half = warp >> 2;
-    const int row = quarter * 32 + lane;
-    const int qr = row / G, hr = row % G;
+    // ------------------------------------------- softmax warpgroup of Q tile tq
+    const int tq = warp >> 2, quarter = warp & 3;
+    const int row = quarter * 32 + lane;              // row of the Q tile = tensor-memory lane
+    const int qr = tq * QT1 + row / G, hr = row % G;  // query of the CTA, head of the group
     const bool rv = qr < c.nq;
     const int64_t t = c.t0 + qr;
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     const int64_t hrow = (c.q0 + qr) * a.Hq + (int64_t)g * G + hr;
     const int64_t t_min = c.t0;  // every row sees at least keys [0, t0]
-    // Softmax in base 2: with c2 = scale * log2(e), exp(scale*s - m) = 2^(c2*s - m2)
-    // where m2 = m * log2(e); the row statistics (m2, l) are kept in that form.
-    // Pass B folds the normalisation into the exponent: P = 2^(c2*s - (m2 + log2 l)).
-    const float c2 = a.scale * 1.4426950408889634f;
-    float m = -INFINITY, l = 0.f, mb = 0.f;
-    if (OUT && rv) {
-      m = a.ml[hrow * 2];
-      l = a.ml[hrow * 2 + 1];
-      mb = m + log2f(l);  // l >= 1: the row's largest logit contributes 1
-    }
     float* srow = a.scores + ((c.q0 + qr) * a.Hkv + g) * a.stride;
     const bool v4 = ((reinterpret_cast<uintptr_t>(a.scores) | ((uintptr_t)a.stride * 4)) & 15) == 0;
-    // Every tcgen05.ld/st and full-mask shuffle below must be reached by the
-    // whole warp: the branches around them use warp-uniform conditions only.
+    // Every tcgen05.ld/st and full-mask shuffle below is reached by the whole
+    // warp: the branches around them use warp-uniform conditions only.
     const bool all_rv = __all_sync(0xffffffffu, rv);
+    // Softmax in base 2: with c2 = scale * log2(e), exp(scale*s - m) = 2^(c2*s - m2)
+    // where m2 = m * log2(e); pass B folds the normalisation into the exponent:
+    // P = 2^(c2*s - (m2 + log2 l)).
+    const float c2 = a.scale * 1.4426950408889634f;
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+    // ---- pass A: running max and sum
+    for (int j = 0; j < n; ++j) {
       const int b = j & 1;
-      if (ok && !mbar_wait(&s_full[b], (uint32_t)(j >> 1) & 1u)) {
+      if (ok && !mbar_wait(&sa_full[tq][b], (uint32_t)(j >> 1) & 1u)) {
         record_error(a.err, HS2_ERR_TIMEOUT);
         ok = false;
       }
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok) {
-        // this warp's 64 keys of the tile: k0 .. k0+63
-        const int64_t k0 = (int64_t)j * kTcKeys + half * 64;
-        uint32_t r[2][32];
-        tmem_ld32(trow + b * kTcKeys + half * 64, r[0]);
-        tmem_ld32(trow + b * kTcKeys + half * 64 + 32, r[1]);
-        tmem_wait_ld();
-        auto S = [&](int i) { return __uint_as_float(r[i >> 5][i & 31]); };
-        // MASKED: some key of the 64 lies past some row's position (or rows past the chunk)
-        auto body = [&](auto masked_c) {
-          constexpr bool MASKED = decltype(masked_c)::value;
-          // keys k0 .. k0+nv-1 are visible to this row
-          const int nv = MASKED ? (rv ? (int)max((int64_t)0, min((int64_t)64, t - k0 + 1)) : 0) : 64;
-          auto valid = [nv](int i) { return !MASKED || i < nv; };
-          if (!OUT) {
+#pragma unroll 1
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int64_t k0 = (int64_t)j * kTcKeys + h2 * 64;
+          uint32_t r[2][32];
+          tmem_ld32(trow + 256 * tq + 128 * b + h2 * 64, r[0]);
+          tmem_ld32(trow + 256 * tq + 128 * b + h2 * 64 + 32, r[1]);
+          tmem_wait_ld();
+          auto S = [&](int i) { return __uint_as_float(r[i >> 5][i & 31]); };
+          auto body = [&](auto masked_c) {
+            constexpr bool MASKED = decltype(masked_c)::value;
+            // keys k0 .. k0+nv-1 are visible to this row
+            const int nv = MASKED ? (rv ? (int)max((int64_t)0, min((int64_t)64, t - k0 + 1)) : 0) : 64;
+            auto valid = [nv](int i) { return !MASKED || i < nv; };
             float mx[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
-              mx[i & 7] = fmaxf(mx[i & 7], valid(i) ? S(i) : -INFINITY);
+            for (int i = 0; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], valid(i) ? S(i) : -INFINITY);
             const float cm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
             if (cm != -INFINITY) {
@@ -251,112 +292,110 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                   (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
               m = mn;
             }
-          } else {
-            float p[64];
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-              const float e = ex2_approx(fmaf(S(i), c2, -mb));
-              p[i] = valid(i) ? e : 0.f;
-            }
-            // P (bf16) into this tile's P buffer: 64 keys -> 32 packed columns
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              uint32_t pk[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(p[32 * cc + 2 * i], p[32 * cc + 2 * i + 1]);
-              tmem_st16(trow + kColP + b * (kTcKeys / 2) + half * 32 + cc * 16, pk);
-            }
-            // scores: sum over the G rows of each query (consecutive lanes) by a
-            // reduce-scatter butterfly on both 32-key chunks; each lane ends with
-            // 32/G consecutive keys of each chunk, at offset ``off``
-            int off = 0, n = 32;
-#pragma unroll
-            for (int msk = G / 2; msk >= 1; msk >>= 1) {
-              const bool up = (lane & msk) != 0;
-              n >>= 1;
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                  if (i < n) {
-                    float* q = p + 32 * cc;
-                    const float send = up ? q[i] : q[i + n];
-                    const float keep = up ? q[i + n] : q[i];
-                    q[i] = keep + __shfl_xor_sync(0xffffffffu, send, msk);
-                  }
-                }
-              }
-              if (up) off += n;
-            }
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              const int64_t kc = k0 + 32 * cc + off;
-              if (!MASKED && v4) {
-                float4* dst = reinterpret_cast<float4*>(srow + kc);
-#pragma unroll
-                for (int i = 0; i < 32 / G / 4; ++i)
-                  dst[i] = make_float4(p[32 * cc + 4 * i], p[32 * cc + 4 * i + 1],
-                                       p[32 * cc + 4 * i + 2], p[32 * cc + 4 * i + 3]);
-              } else if (rv) {
-#pragma unroll
-                for (int i = 0; i < 32 / G; ++i)
-                  if (kc + i <= t) srow[kc + i] = p[32 * cc + i];
-              }
-            }
-          }
-        };
-        if (all_rv && k0 + 63 <= t_min) body(std::false_type{});
-        else body(std::true_type{});
+          };
+          if (all_rv && k0 + 63 <= t_min) body(std::false_type{});
+          else body(std::true_type{});
+        }
       }
-      if (OUT) tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(OUT ? &p_full[b] : &s_free[b]);
+      if (lane == 0) mbar_arrive(&sa_free[tq][b]);
     }
-    if (!OUT) {
-      // merge the two column halves' running (m, l) of each row
-      if (half == 1) {
-        half_ml[0][row] = m;
-        half_ml[1][row] = l;
-      }
-      named_barrier_sync(1, 32 * kTcSoftWarps);
-      if (half == 0 && rv) {
-        const float m2 = half_ml[0][row], l2 = half_ml[1][row];
-        const float mm = fmaxf(m, m2);
-        const float ll = (mm == -INFINITY) ? 0.f : l * ex2_approx(m - mm) + l2 * ex2_approx(m2 - mm);
-        a.ml[hrow * 2] = mm;
-        a.ml[hrow * 2 + 1] = ll;
-      }
-    } else {
-      if (ok && !mbar_wait(&o_full, 0)) {
+    const float mb = (rv && l > 0.f) ? m + log2f(l) : 0.f;  // l >= 1 for a visible row
+    // ---- pass B: P, scores, O += P V
+    for (int j = 0; j < n; ++j) {
+      if (ok && !mbar_wait(&sb_full[tq], (uint32_t)j & 1u)) {
         record_error(a.err, HS2_ERR_TIMEOUT);
         ok = false;
       }
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      bf16* O = static_cast<bf16*>(a.O);
+      if (ok) {
 #pragma unroll 1
-      for (int cc = 0; cc < 2 && ok; ++cc) {
-        const int ch = half * 2 + cc;
-        uint32_t r[32];
-        tmem_ld32(trow + kColO + ch * 32, r);
-        tmem_wait_ld();
-        if (rv) {
-          uint32_t pk[16];
+        for (int cc = 0; cc < 4; ++cc) {  // 32 keys at a time; their P goes behind them
+          const int64_t kc = (int64_t)j * kTcKeys + cc * 32;
+          uint32_t r[32];
+          tmem_ld32(trow + 128 * tq + cc * 32, r);
+          tmem_wait_ld();
+          auto body = [&](auto masked_c) {
+            constexpr bool MASKED = decltype(masked_c)::value;
+            const int nv = MASKED ? (rv ? (int)max((int64_t)0, min((int64_t)32, t - kc + 1)) : 0) : 32;
+            float p[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          uint4* dst = reinterpret_cast<uint4*>(O + hrow * kD + ch * 32);
+            for (int i = 0; i < 32; ++i) {
+              const float e = ex2_approx(fmaf(__uint_as_float(r[i]), c2, -mb));
+              p[i] = (!MASKED || i < nv) ? e : 0.f;
+            }
+            uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(p[2 * i], p[2 * i + 1]);
+            tmem_st16(trow + 128 * tq + cc * 16, pk);
+            // scores: sum over the G rows of each query (consecutive lanes) by a
+            // reduce-scatter butterfly; each lane ends with 32/G consecutive keys
+            int off = 0, nn = 32;
+#pragma unroll
+            for (int msk = G / 2; msk >= 1; msk >>= 1) {
+              const bool up = (lane & msk) != 0;
+              nn >>= 1;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                if (i < nn) {
+                  const float send = up ? p[i] : p[i + nn];
+                  const float keep = up ? p[i + nn] : p[i];
+                  p[i] = keep + __shfl_xor_sync(0xffffffffu, send, msk);
+                }
+              }
+              if (up) off += nn;
+            }
+            const int64_t ks = kc + off;
+            if (!MASKED && v4) {
+              float4* dst = reinterpret_cast<float4*>(srow + ks);
+#pragma unroll
+              for (int i = 0; i < 32 / G / 4; ++i)
+                dst[i] = make_float4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            } else if (rv) {
+#pragma unroll
+              for (int i = 0; i < 32 / G; ++i)
+                if (ks + i <= t) srow[ks + i] = p[i];
+            }
+          };
+          if (all_rv && kc + 31 <= t_min) body(std::false_type{});
+          else body(std::true_type{});
         }
       }
+      tmem_wait_st();
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pb_full[tq]);
     }
+    // ---- O of this row: bf16 out of tensor memory
+    if (ok && !mbar_wait(&o_full, 0)) {
+      record_error(a.err, HS2_ERR_TIMEOUT);
+      ok = false;
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    bf16* O = static_cast<bf16*>(a.O);
+#pragma unroll 1
+    for (int ch = 0; ch < 4 && ok; ++ch) {
+      uint32_t r[32];
+      tmem_ld32(trow + 256 + 128 * tq + ch * 32, r);
+      tmem_wait_ld();
+      if (rv) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        uint4* dst = reinterpret_cast<uint4*>(O + hrow * kD + ch * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
+    }
+    tc_fence_before();
   }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 

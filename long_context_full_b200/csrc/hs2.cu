@@ -71,11 +71,7 @@ std::mutex g_dev_mu;
 
 template <int G>
 cudaError_t set_chunk_tc_smem() {
-  cudaError_t e = cudaFuncSetAttribute(k_chunk_tc<false, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)chunk_tc_smem<false>());
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_chunk_tc<true, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)chunk_tc_smem<true>());
+  return cudaFuncSetAttribute(k_chunk_tc<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chunk_tc_smem());
 }
 
 hs2_status device_info(DeviceInfo** out) {
@@ -297,8 +293,7 @@ hs2_status check_chunk(const hs2_problem* p) {
 template <int G>
 void launch_chunk_tc(dim3 grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
                      const CUtensorMap& mv, const ChunkArgs& a) {
-  launch(k_chunk_tc<false, G>, dim3(grid), dim3(kTcThreads), chunk_tc_smem<false>(), st, 0, mq, mk, mv, a);
-  launch(k_chunk_tc<true, G>, dim3(grid), dim3(kTcThreads), chunk_tc_smem<true>(), st, 0, mq, mk, mv, a);
+  launch(k_chunk_tc<G>, grid, dim3(kTcThreads), chunk_tc_smem(), st, 0, mq, mk, mv, a);
 }
 
 template <int GP>
@@ -319,9 +314,9 @@ hs2_status run_chunk(const hs2_problem* p, const DeviceInfo& dev, const void* Q,
   a.total_q = p->total_q; a.total_kv = p->total_kv; a.scale = p->scale;
   a.O = O; a.ml = pl.ml; a.scores = scores; a.stride = stride; a.err = dev.err;
   if (p->dtype == HS2_BF16) {
-    a.QT = kTcRows / a.G;
+    a.QT = kTcQTiles * kTcRows / a.G;  // queries per CTA (two Q tiles)
     CUtensorMap mq, mk, mv;
-    if (encode_map3(&mq, Q, p->total_q, p->Hq, a.G, a.QT) != HS2_OK ||
+    if (encode_map3(&mq, Q, p->total_q, p->Hq, a.G, kTcRows / a.G) != HS2_OK ||
         encode_map3(&mk, K, p->total_kv, p->Hkv, 1, kTcKeys) != HS2_OK ||
         encode_map3(&mv, V, p->total_kv, p->Hkv, 1, kTcKeys) != HS2_OK)
       return HS2_ERR_CUDA;
