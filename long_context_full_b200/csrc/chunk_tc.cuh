@@ -25,8 +25,8 @@
 // the TMA loads (Q once; K and V through separate two-stage rings); warp 9
 // issues the MMAs from one thread.  Tensor memory (512 columns): pass A, the S
 // buffers (tile t, buffer b) at 256t + 128b; pass B, S_t/P_t at 128t and O_t
-// at 256 + 128t.  Before S_t of the next key tile overwrites P_t, the MMA
-// thread waits for the commit of the O_t += P_t V that reads it.
+// at 256 + 128t.  S_t of the next key tile is issued right after the
+// O_t += P_t V that reads P_t: tcgen05.mma from one thread execute in order.
 #pragma once
 
 #include <type_traits>
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t k_full[kTcStages], k_empty[kTcStages];
   __shared__ __align__(8) uint64_t v_full[kTcStages], v_empty[kTcStages];
   __shared__ __align__(8) uint64_t sa_full[2][2], sa_free[2][2];  // pass A: [Q tile][S buffer]
-  __shared__ __align__(8) uint64_t sb_full[2], pb_full[2], pv_done[2], o_full;  // pass B: [Q tile]
+  __shared__ __align__(8) uint64_t sb_full[2], pb_full[2], o_full;  // pass B: [Q tile]
   __shared__ uint32_t tmem_base_sh;
 
   ChTile c;
@@ -89,7 +89,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       mbar_init(&sb_full[t], 1);
       mbar_init(&pb_full[t], 4);
-      mbar_init(&pv_done[t], 1);
     }
     mbar_init(&o_full, 1);
     fence_mbar_init();
@@ -207,11 +206,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             umma_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8,
                     umma_desc_sw128(vb + kk * 2048, kTcTileBytes / 2, 1024), idesc_o,
                     (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&pv_done[t]);
           if (t == 1) umma_commit(&v_empty[vst]);
           if (j + 1 < n) {
-            // P_t is read by the MMAs just issued; S_t of the next tile overwrites it
-            if (!(ok = mbar_wait(&pv_done[t], (uint32_t)j & 1u))) break;
+            // S_t of the next tile overwrites P_t, which the MMAs just issued
+            // read: tcgen05.mma from one thread execute in issue order
             if (t == 0 && !(ok = kwait(kf))) break;
             tc_fence_after();
             mma_s(128 * t, t, kf % kTcStages);
@@ -220,11 +218,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      umma_commit(&o_full);
-      // the last commits have arrived before the CTA exits
-      if (ok && n > 0)
-        for (int t = 0; t < 2; ++t)
-          if (!mbar_wait(&pv_done[t], (uint32_t)(n - 1) & 1u)) ok = false;
+      umma_commit(&o_full);  // every MMA of the CTA (the softmax warps wait for it)
       if (!ok) record_error(a.err, HS2_ERR_TIMEOUT);
     }
   } else {
@@ -258,51 +252,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok) {
-#pragma unroll 1
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int64_t k0 = (int64_t)j * kTcKeys + h2 * 64;
-          uint32_t r[2][32];
-          tmem_ld32(trow + 256 * tq + 128 * b + h2 * 64, r[0]);
-          tmem_ld32(trow + 256 * tq + 128 * b + h2 * 64 + 32, r[1]);
-          tmem_wait_ld();
-          auto S = [&](int i) { return __uint_as_float(r[i >> 5][i & 31]); };
-          auto body = [&](auto masked_c) {
-            constexpr bool MASKED = decltype(masked_c)::value;
-            // keys k0 .. k0+nv-1 are visible to this row
-            const int nv = MASKED ? (rv ? (int)max((int64_t)0, min((int64_t)64, t - k0 + 1)) : 0) : 64;
-            auto valid = [nv](int i) { return !MASKED || i < nv; };
-            float mx[8];
+        // the whole 128-key row of S at once: one wait, 128-wide independent work
+        const int64_t k0 = (int64_t)j * kTcKeys;
+        uint32_t r[4][32];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+        for (int q = 0; q < 4; ++q) tmem_ld32(trow + 256 * tq + 128 * b + 32 * q, r[q]);
+        tmem_wait_ld();
+        auto S = [&](int i) { return __uint_as_float(r[i >> 5][i & 31]); };
+        auto body = [&](auto masked_c) {
+          constexpr bool MASKED = decltype(masked_c)::value;
+          // keys k0 .. k0+nv-1 are visible to this row
+          const int nv = MASKED ? (rv ? (int)max((int64_t)0, min((int64_t)kTcKeys, t - k0 + 1)) : 0) : kTcKeys;
+          auto valid = [nv](int i) { return !MASKED || i < nv; };
+          float mx[8];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], valid(i) ? S(i) : -INFINITY);
-            const float cm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            if (cm != -INFINITY) {
-              const float mn = fmaxf(m, cm * c2);
-              float sm[8];
+          for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
 #pragma unroll
-              for (int u = 0; u < 8; ++u) sm[u] = 0.f;
+          for (int i = 0; i < kTcKeys; ++i) mx[i & 7] = fmaxf(mx[i & 7], valid(i) ? S(i) : -INFINITY);
+          const float cm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          if (cm != -INFINITY) {
+            const float mn = fmaxf(m, cm * c2);
+            float sm[8];
 #pragma unroll
-              for (int i = 0; i < 64; ++i) {
-                const float e = ex2_approx(fmaf(S(i), c2, -mn));
-                sm[i & 7] += valid(i) ? e : 0.f;
-              }
-              l = l * ex2_approx(m - mn) +
-                  (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
-              m = mn;
+            for (int u = 0; u < 8; ++u) sm[u] = 0.f;
+#pragma unroll
+            for (int i = 0; i < kTcKeys; ++i) {
+              const float e = ex2_approx(fmaf(S(i), c2, -mn));
+              sm[i & 7] += valid(i) ? e : 0.f;
             }
-          };
-          if (all_rv && k0 + 63 <= t_min) body(std::false_type{});
-          else body(std::true_type{});
-        }
+            l = l * ex2_approx(m - mn) +
+                (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+            m = mn;
+          }
+        };
+        if (all_rv && k0 + kTcKeys - 1 <= t_min) body(std::false_type{});
+        else body(std::true_type{});
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sa_free[tq][b]);
     }
     const float mb = (rv && l > 0.f) ? m + log2f(l) : 0.f;  // l >= 1 for a visible row
-    // ---- pass B: P, scores, O += P V
+    // ---- pass B: P (handed to the MMA warp first), then the scores
     for (int j = 0; j < n; ++j) {
       if (ok && !mbar_wait(&sb_full[tq], (uint32_t)j & 1u)) {
         record_error(a.err, HS2_ERR_TIMEOUT);
@@ -310,63 +302,77 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
+      const int64_t k0 = (int64_t)j * kTcKeys;
+      const bool full = all_rv && k0 + kTcKeys - 1 <= t_min;  // no key of the tile is masked
+      // keys k0 .. k0+nv-1 are visible to this row
+      const int nv = full ? kTcKeys : (rv ? (int)max((int64_t)0, min((int64_t)kTcKeys, t - k0 + 1)) : 0);
+      float p[4][32];
       if (ok) {
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {  // 32 keys at a time; their P goes behind them
-          const int64_t kc = (int64_t)j * kTcKeys + cc * 32;
-          uint32_t r[32];
-          tmem_ld32(trow + 128 * tq + cc * 32, r);
-          tmem_wait_ld();
-          auto body = [&](auto masked_c) {
-            constexpr bool MASKED = decltype(masked_c)::value;
-            const int nv = MASKED ? (rv ? (int)max((int64_t)0, min((int64_t)32, t - kc + 1)) : 0) : 32;
-            float p[32];
+        // the whole 128-key row of S at once, then P (bf16) into the first 64
+        // columns, which have been read
+        uint32_t r[4][32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float e = ex2_approx(fmaf(__uint_as_float(r[i]), c2, -mb));
-              p[i] = (!MASKED || i < nv) ? e : 0.f;
-            }
-            uint32_t pk[16];
+        for (int q = 0; q < 4; ++q) tmem_ld32(trow + 128 * tq + 32 * q, r[q]);
+        tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(p[2 * i], p[2 * i + 1]);
-            tmem_st16(trow + 128 * tq + cc * 16, pk);
-            // scores: sum over the G rows of each query (consecutive lanes) by a
-            // reduce-scatter butterfly; each lane ends with 32/G consecutive keys
-            int off = 0, nn = 32;
+        for (int q = 0; q < 4; ++q) {
 #pragma unroll
-            for (int msk = G / 2; msk >= 1; msk >>= 1) {
-              const bool up = (lane & msk) != 0;
-              nn >>= 1;
+          for (int i = 0; i < 32; ++i) {
+            const float e = ex2_approx(fmaf(__uint_as_float(r[q][i]), c2, -mb));
+            p[q][i] = (full || 32 * q + i < nv) ? e : 0.f;
+          }
+          uint32_t pk[16];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                if (i < nn) {
-                  const float send = up ? p[i] : p[i + nn];
-                  const float keep = up ? p[i + nn] : p[i];
-                  p[i] = keep + __shfl_xor_sync(0xffffffffu, send, msk);
-                }
-              }
-              if (up) off += nn;
-            }
-            const int64_t ks = kc + off;
-            if (!MASKED && v4) {
-              float4* dst = reinterpret_cast<float4*>(srow + ks);
-#pragma unroll
-              for (int i = 0; i < 32 / G / 4; ++i)
-                dst[i] = make_float4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-            } else if (rv) {
-#pragma unroll
-              for (int i = 0; i < 32 / G; ++i)
-                if (ks + i <= t) srow[ks + i] = p[i];
-            }
-          };
-          if (all_rv && kc + 31 <= t_min) body(std::false_type{});
-          else body(std::true_type{});
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(p[q][2 * i], p[q][2 * i + 1]);
+          tmem_st16(trow + 128 * tq + 16 * q, pk);
         }
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&pb_full[tq]);
+      if (ok) {
+        // scores: sum over the G rows of each query (consecutive lanes) by a
+        // reduce-scatter butterfly, two 32-key chunks at a time; each lane ends
+        // with 32/G consecutive keys of each chunk, at offset ``off``
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          int off = 0, nn = 32;
+#pragma unroll
+          for (int msk = G / 2; msk >= 1; msk >>= 1) {
+            const bool up = (lane & msk) != 0;
+            nn >>= 1;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+#pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                if (i < nn) {
+                  float* q = p[2 * hh + cc];
+                  const float send = up ? q[i] : q[i + nn];
+                  const float keep = up ? q[i + nn] : q[i];
+                  q[i] = keep + __shfl_xor_sync(0xffffffffu, send, msk);
+                }
+              }
+            }
+            if (up) off += nn;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const float* q = p[2 * hh + cc];
+            const int64_t ks = k0 + 64 * hh + 32 * cc + off;
+            if (full && v4) {
+              float4* dst = reinterpret_cast<float4*>(srow + ks);
+#pragma unroll
+              for (int i = 0; i < 32 / G / 4; ++i)
+                dst[i] = make_float4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]);
+            } else if (rv) {
+#pragma unroll
+              for (int i = 0; i < 32 / G; ++i)
+                if (ks + i <= t) srow[ks + i] = q[i];
+            }
+          }
+        }
+      }
     }
     // ---- O of this row: bf16 out of tensor memory
     if (ok && !mbar_wait(&o_full, 0)) {
