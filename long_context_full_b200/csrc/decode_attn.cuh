@@ -418,6 +418,7 @@ __global__ void __launch_bounds__(kD) k_decode_combine(const __grid_constant__ D
 // of the tile for every KV head; the writes are coalesced along j.
 // ----------------------------------------------------------------------------
 constexpr int kFinKeys = 128;
+constexpr float kLog2e = 1.4426950408889634f;
 
 // Tile -> (sequence, first key); tiles cover ceil(max_len / kFinKeys) blocks
 // of every sequence, empty ones are skipped.
@@ -485,7 +486,11 @@ __global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_const
       if (q0 < 0 || q0 >= a.total_q || kb < 0 || kb + N > a.total_kv || N > stride) {
         if (threadIdx.x == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
       } else {
-        for (int i = threadIdx.x; i < 2 * Hq; i += kFinKeys) fst[i] = __ldg(ml + q0 * Hq * 2 + i);
+        // (m_h, 1/l_h) -> (m_h * log2 e, 1/l_h): exp(x - m) = 2^(x log2 e - m log2 e)
+        for (int i = threadIdx.x; i < 2 * Hq; i += kFinKeys) {
+          const float v = __ldg(ml + q0 * Hq * 2 + i);
+          fst[i] = (i & 1) ? v : v * 1.4426950408889634f;
+        }
         cp_async_wait_prev();  // this tile's copy has landed (the next may be in flight)
         __syncthreads();
         const int kj = threadIdx.x;
@@ -496,14 +501,14 @@ __global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_const
             if (vec4) {  // 16-byte reads: the row pitch of 9 x 16 bytes spreads 8 lanes over all banks
               for (int h = g * a.G; h < (g + 1) * a.G; h += 4) {
                 const float4 v = *reinterpret_cast<const float4*>(x + h);
-                sc = fmaf(expf(v.x - fst[2 * h]), fst[2 * h + 1], sc);
-                sc = fmaf(expf(v.y - fst[2 * h + 2]), fst[2 * h + 3], sc);
-                sc = fmaf(expf(v.z - fst[2 * h + 4]), fst[2 * h + 5], sc);
-                sc = fmaf(expf(v.w - fst[2 * h + 6]), fst[2 * h + 7], sc);
+                sc = fmaf(ex2_approx(fmaf(v.x, kLog2e, -fst[2 * h])), fst[2 * h + 1], sc);
+                sc = fmaf(ex2_approx(fmaf(v.y, kLog2e, -fst[2 * h + 2])), fst[2 * h + 3], sc);
+                sc = fmaf(ex2_approx(fmaf(v.z, kLog2e, -fst[2 * h + 4])), fst[2 * h + 5], sc);
+                sc = fmaf(ex2_approx(fmaf(v.w, kLog2e, -fst[2 * h + 6])), fst[2 * h + 7], sc);
               }
             } else {
               for (int h = g * a.G; h < (g + 1) * a.G; ++h)
-                sc = fmaf(expf(x[h] - fst[2 * h]), fst[2 * h + 1], sc);
+                sc = fmaf(ex2_approx(fmaf(x[h], kLog2e, -fst[2 * h])), fst[2 * h + 1], sc);
             }
             scores[(q0 * a.Hkv + g) * stride + j0 + kj] = sc;
           }

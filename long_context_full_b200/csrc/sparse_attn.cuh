@@ -188,62 +188,72 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
       spos[row] = row < pn ? sparse_pos(a, s, p0 + row, true) : -1;
     __syncthreads();
     // gather: 16-byte cp.async per (row, chunk), 16 chunks of K and 16 of V per
-    // row; rows past pn or with an invalid index are zero-filled (no read)
-    for (int i = threadIdx.x; i < ntile * 16 * 32; i += blockDim.x) {
-      const int row = i >> 5, ch = i & 31, c16 = ch & 15;
-      const int64_t pos = spos[row];
-      const bool ok = pos >= 0;
-      const bf16* base = ch < 16 ? K : V;
-      const bf16* src = ok ? base + ((s.kv_start + pos) * a.Hkv + s.g) * kD + c16 * 8 : base;
-      uint8_t* dst = (ch < 16 ? sK : sV) + (size_t)row * kSpRowBytes + c16 * 16;
-      cp_async16(dst, src, ok ? 16 : 0);
+    // row; rows past pn or with an invalid index are zero-filled (no read).  Two
+    // copy groups: the first half of the slices is scored while the second
+    // half is still in flight.
+    const int nA = (ntile + 1) / 2;
+    for (int grp = 0; grp < 2; ++grp) {
+      const int lo = grp == 0 ? 0 : nA * 16 * 32, hi = grp == 0 ? nA * 16 * 32 : ntile * 16 * 32;
+      for (int i = lo + (int)threadIdx.x; i < hi; i += blockDim.x) {
+        const int row = i >> 5, ch = i & 31, c16 = ch & 15;
+        const int64_t pos = spos[row];
+        const bool ok = pos >= 0;
+        const bf16* base = ch < 16 ? K : V;
+        const bf16* src = ok ? base + ((s.kv_start + pos) * a.Hkv + s.g) * kD + c16 * 8 : base;
+        uint8_t* dst = (ch < 16 ? sK : sV) + (size_t)row * kSpRowBytes + c16 * 16;
+        cp_async16(dst, src, ok ? 16 : 0);
+      }
+      cp_async_commit();
     }
-    cp_async_wait_all();
-    __syncthreads();
-    for (int st = warp; st < ntile; st += kSpWarps) {
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-      {
-        const int row = st * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+    for (int half = 0; half < 2; ++half) {
+      if (half == 0) cp_async_wait_prev();
+      else cp_async_wait_all_groups();
+      __syncthreads();
+      for (int st = (half == 0 ? 0 : nA) + warp; st < (half == 0 ? nA : ntile); st += kSpWarps) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const int row = st * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const int chunk = kk * 2 + (lane >> 4);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(a0, a1, a2, a3, skb + row * kSpRowBytes + chunk * 16);
-          mma_bf16(c, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+          for (int kk = 0; kk < 8; ++kk) {
+            const int chunk = kk * 2 + (lane >> 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(a0, a1, a2, a3, skb + row * kSpRowBytes + chunk * 16);
+            mma_bf16(c, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+          }
         }
-      }
-      const int ilo = st * 16 + r, ihi = ilo + 8;
-      const bool vlo = spos[ilo] >= 0, vhi = spos[ihi] >= 0;
-      const float x0 = vlo ? c[0] * a.scale : NEG, x1 = vlo ? c[1] * a.scale : NEG;
-      const float x2 = vhi ? c[2] * a.scale : NEG, x3 = vhi ? c[3] * a.scale : NEG;
-      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+        const int ilo = st * 16 + r, ihi = ilo + 8;
+        const bool vlo = spos[ilo] >= 0, vhi = spos[ihi] >= 0;
+        const float x0 = vlo ? c[0] * a.scale : NEG, x1 = vlo ? c[1] * a.scale : NEG;
+        const float x2 = vhi ? c[2] * a.scale : NEG, x3 = vhi ? c[3] * a.scale : NEG;
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float al0 = (mn0 == NEG) ? 1.f : exp_shift(m0, mn0);
-      const float al1 = (mn1 == NEG) ? 1.f : exp_shift(m1, mn1);
-      const float p0v = exp_shift(x0, mn0), p1v = exp_shift(x1, mn1);
-      const float p2v = exp_shift(x2, mn0), p3v = exp_shift(x3, mn1);
-      l0 = l0 * al0 + (p0v + p2v);
-      l1 = l1 * al1 + (p1v + p3v);
-      m0 = mn0;
-      m1 = mn1;
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float al0 = (mn0 == NEG) ? 1.f : exp_shift(m0, mn0);
+        const float al1 = (mn1 == NEG) ? 1.f : exp_shift(m1, mn1);
+        const float p0v = exp_shift(x0, mn0), p1v = exp_shift(x1, mn1);
+        const float p2v = exp_shift(x2, mn0), p3v = exp_shift(x3, mn1);
+        l0 = l0 * al0 + (p0v + p2v);
+        l1 = l1 * al1 + (p1v + p3v);
+        m0 = mn0;
+        m1 = mn1;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        o[i][0] *= al0; o[i][1] *= al1; o[i][2] *= al0; o[i][3] *= al1;
-      }
-      const uint32_t b0 = movmatrix_t(pack_bf16(p0v, p1v));
-      const uint32_t b1 = movmatrix_t(pack_bf16(p2v, p3v));
-      const int row = st * 16 + ((lane >> 4) & 1) * 8 + (lane & 7);
+        for (int i = 0; i < 8; ++i) {
+          o[i][0] *= al0; o[i][1] *= al1; o[i][2] *= al0; o[i][3] *= al1;
+        }
+        const uint32_t b0 = movmatrix_t(pack_bf16(p0v, p1v));
+        const uint32_t b1 = movmatrix_t(pack_bf16(p2v, p3v));
+        const int row = st * 16 + ((lane >> 4) & 1) * 8 + (lane & 7);
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const int chunk = mt * 2 + ((lane >> 3) & 1);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(a0, a1, a2, a3, svb + row * kSpRowBytes + chunk * 16);
-        mma_bf16(o[mt], a0, a1, a2, a3, b0, b1);
+        for (int mt = 0; mt < 8; ++mt) {
+          const int chunk = mt * 2 + ((lane >> 3) & 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(a0, a1, a2, a3, svb + row * kSpRowBytes + chunk * 16);
+          mma_bf16(o[mt], a0, a1, a2, a3, b0, b1);
+        }
       }
     }
     __syncthreads();  // the next piece overwrites the staged rows
