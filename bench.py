@@ -53,7 +53,8 @@ def parse():
     ap.add_argument("--context", type=int, default=CONTEXT,
                     help="cached tokens per sequence (smaller only for profiling captures)")
     ap.add_argument("--workload", default="decode_b8_128k",
-                    choices=["decode_b8_128k", "needle_1m", "ragged_16", "chunk_256k"],
+                    choices=["decode_b8_128k", "needle_1m", "ragged_16", "chunk_256k",
+                             "multiblock_4x_decode_b8_128k"],
                     help="other shapes of the pages' workloads (one GPU); the default is the "
                          "benchmark line")
     return ap.parse_args()
@@ -310,6 +311,107 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
+def run_multiblock(args, local: int, n_blocks: int = 4):
+    """A decode step through ``n_blocks`` Hybrid Blocks, each with its own
+    8 x 131072-token cache (8 GiB of K/V in all), replayed as one CUDA graph:
+    per block, the new token's K/V appended, full attention with scores, top-k
+    selection and 4 sparse layers.  Throughput = the 8 query tokens of the step
+    / step time.  End to end: the step's inputs (queries of every layer and the
+    new K/V rows of every block) copied from pinned host memory and the last
+    sparse layer's output of every block read back; the caches stay resident."""
+    import torch
+    import synth
+    from long_context_full_b200 import hs2
+    from long_context_full_b200.multiblock import BlockInputs, MultiBlockDecodeStep
+
+    ws = [synth.decode_128k(batch=BATCH, first_seq=BATCH * i, context=CONTEXT) for i in range(n_blocks)]
+    rng = np.random.default_rng(2026)
+    news = [(synth.f32_to_bf16_bits(rng.standard_normal((BATCH, HKV, D)).astype(np.float32)),
+             synth.f32_to_bf16_bits(rng.standard_normal((BATCH, HKV, D)).astype(np.float32)))
+            for _ in range(n_blocks)]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    ins = [BlockInputs(dev(w.k), dev(w.v), dev(kn), dev(vn), dev(w.q), [dev(x) for x in w.q_layers])
+           for w, (kn, vn) in zip(ws, news)]
+    w0 = ws[0]
+    mb = MultiBlockDecodeStep(n_blocks, w0.Hq, w0.Hkv, w0.D, torch.bfloat16, w0.q_lens, w0.kv_lens,
+                              w0.n_layers, k=TOPK, window=WINDOW)
+    outs = mb.capture(ins)
+    for _ in range(max(3, args.warmup)):
+        mb.replay()
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    stream = torch.cuda.current_stream()
+    Kst = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(stream)
+    for _ in range(Kst):
+        mb.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    ms_step = start.elapsed_time(end) / Kst
+    value = BATCH / (ms_step * 1e-3)
+    ab = workload_accounting(w0, w0.n_layers)
+    append_bytes = 2 * 2 * BATCH * HKV * D * 2  # new rows read and written, K and V
+    step_bytes = n_blocks * (ab["step"] + append_bytes)
+    hbm, hbm_kind = peaks()
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9
+
+    # end to end: inputs from pinned host memory, outputs back, graph replay between
+    hin = [(pin(w.q), [pin(x) for x in w.q_layers], pin(kn), pin(vn)) for w, (kn, vn) in zip(ws, news)]
+    dpairs = []
+    for x, (hq, hql, hkn, hvn) in zip(ins, hin):
+        dpairs += [(x.Q, hq), (x.K_new, hkn), (x.V_new, hvn)] + list(zip(x.Q_layers, hql))
+    douts = [o.O_layers[-1] for o in outs]
+    houts = [torch.empty_like(o, device="cpu").pin_memory() for o in douts]
+    h2d = sum(h.numel() * h.element_size() for _, h in dpairs)
+    d2h = sum(h.numel() * h.element_size() for h in houts)
+
+    def e2e_step():
+        for d_, h_ in dpairs:
+            d_.copy_(h_, non_blocking=True)
+        mb.replay()
+        for h_, d_ in zip(houts, douts):
+            h_.copy_(d_, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    E = max(1, min(args.e2e_steps, Kst))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_value = BATCH * E / (e0.elapsed_time(e1) * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": Kst,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V, Philox streams)",
+        "config": {"workload": f"multiblock_{n_blocks}x_decode_b8_128k_bf16 (CUDA graph)",
+                   "blocks": n_blocks, "query_tokens_per_gpu": BATCH, "context": CONTEXT,
+                   "Hq": HQ, "Hkv": HKV, "D": D, "k": TOPK, "window": WINDOW,
+                   "reuse_layers": w0.n_layers,
+                   "l2": f"inputs larger than L2: {n_blocks * ab['kv'] / 2**30:.2f} GiB of K/V per step",
+                   "parallelism": "dp1"},
+        "roofline": {"kernel": "whole step (all blocks)", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "peak_kind": hbm_kind,
+                     "traffic": None, "algorithmic_bytes": step_bytes},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": E},
+        "gpu_launches": Kst * mb.launches_per_step(),
+        "clocks": clk,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
@@ -330,6 +432,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     hs2.load()
+    if args.workload == "multiblock_4x_decode_b8_128k":
+        if world > 1:
+            raise SystemExit("--workload other than the default runs on one GPU")
+        return run_multiblock(args, local)
 
     batch, context = args.batch, args.context
     if args.workload == "decode_b8_128k":

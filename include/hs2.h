@@ -22,6 +22,8 @@
  *   hs2_sparse_attn       one sparse layer over the selected rows (call once
  *                         per reuse layer, each with its own queries)
  *   hs2_block_select      (comparison path) first-generation block selection
+ * and, before them in a decode step, hs2_kv_append (the new tokens' K/V rows
+ * written into the cache).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -177,6 +179,22 @@ hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K,
                            const void* V, const int32_t* idx, const int32_t* count,
                            int32_t idx_stride, void* O_l, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * hs2_kv_append - writes the K/V rows of a step's new tokens into the KV cache
+ * that the full-attention layer produces and its sparse layers reuse ([HT]
+ * "Two-Level KV Sharing"; [OH]: decoding extends the cache a token at a time).
+ * Each new token's key goes to its own cache position: query row i of sequence
+ * b (position t = N_b - Tq_b + i) writes K[kv_offsets[b] + t] and
+ * V[kv_offsets[b] + t], all Hkv heads, which is where the attention calls of
+ * the same step read it (the query's own key is in the cache).
+ * K_new, V_new [total_q, Hkv, D]: the new rows (dtype of the problem).
+ * K, V [total_kv, Hkv, D]: the cache, updated in place; no other row changes.
+ * Needs no workspace.  A position outside the cache (offsets that disagree
+ * with the host totals) is recorded as HS2_ERR_DEVICE_INPUT and skipped.
+ */
+hs2_status hs2_kv_append(const hs2_problem* p, const void* K_new, const void* V_new, void* K,
+                         void* V, void* stream);
 
 /* ---------------------------------------------------------------------------
  * hs2_block_select_noalloc - hs2_block_select for callers that cannot give

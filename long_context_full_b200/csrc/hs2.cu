@@ -12,6 +12,7 @@
 #include "hs2.h"
 #include "decode_attn.cuh"
 #include "select.cuh"
+#include "kv_append.cuh"
 #include "sparse_attn.cuh"
 #include "chunk_attn.cuh"
 #include "chunk_tc.cuh"
@@ -617,6 +618,32 @@ const char* hs2_status_string(hs2_status s) {
     case HS2_ERR_DEVICE_INPUT: return "device found inputs that break the contract";
   }
   return "unknown status";
+}
+
+hs2_status hs2_kv_append(const hs2_problem* p, const void* K_new, const void* V_new, void* K,
+                         void* V, void* stream) {
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (p->total_q == 0) return HS2_OK;
+  if (!K_new || !V_new || !K || !V) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(K_new) || !aligned16(V_new) || !aligned16(K) || !aligned16(V)) return HS2_ERR_INVALID_ARG;
+  if (p->total_q > p->total_kv) return HS2_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != HS2_OK) return s;
+  const int64_t warps = p->total_q * p->Hkv;
+  const unsigned grid = (unsigned)((warps * 32 + kAppendThreads - 1) / kAppendThreads);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint8_t* kn = static_cast<const uint8_t*>(K_new);
+  const uint8_t* vn = static_cast<const uint8_t*>(V_new);
+  uint8_t* k = static_cast<uint8_t*>(K);
+  uint8_t* v = static_cast<uint8_t*>(V);
+  if (p->dtype == HS2_BF16)
+    launch(k_kv_append<kD * 2>, dim3(grid), dim3(kAppendThreads), 0, st, 0, kn, vn, k, v, p->q_offsets,
+           p->kv_offsets, p->B, p->Hkv, p->total_q, p->total_kv, dev->err);
+  else
+    launch(k_kv_append<kD * 4>, dim3(grid), dim3(kAppendThreads), 0, st, 0, kn, vn, k, v, p->q_offsets,
+           p->kv_offsets, p->B, p->Hkv, p->total_q, p->total_kv, dev->err);
+  return launch_status();
 }
 
 int32_t hs2_version(void) { return (0 << 16) | 1; }

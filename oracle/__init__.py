@@ -31,16 +31,23 @@ state.  Sources (page title, then section):
   index set: softmax attention restricted to the selected rows.  "Xiaomi
   Unveils HySparse2 for Faster Long-Context AI", sections "Two-Level KV
   Sharing" (KV Reuse) and "Token-Level Selection and Unified Local Access".
+* ``kv_append``            - a step's new K/V rows written into the cache at the
+  tokens' own positions, the cache each Full Attention layer of the
+  Cross-Decoder owns.  "Xiaomi Unveils HySparse2 for Faster Long-Context AI",
+  section "Two-Level KV Sharing" (KV Bridging, KV Reuse).
 
-Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
-invariants and brute force on tiny inputs.
+Every function is pinned by ``tests/test_oracle_pins.py`` (``kv_append`` by
+``tests/test_kv_append_pins.py``) against closed forms, invariants and brute
+force on tiny inputs.
 """
 from .attention import (full_attention_row, selection_scores, sparse_attention_row,
                         run_full_attention, run_sparse_attention)
 from .selection import topk_select, block_select, candidate_count, window_range
+from .cache import kv_append
 
 __all__ = [
     "full_attention_row", "selection_scores", "sparse_attention_row",
     "run_full_attention", "run_sparse_attention",
     "topk_select", "block_select", "candidate_count", "window_range",
+    "kv_append",
 ]
