@@ -54,7 +54,7 @@ def parse():
                     help="cached tokens per sequence (smaller only for profiling captures)")
     ap.add_argument("--workload", default="decode_b8_128k",
                     choices=["decode_b8_128k", "needle_1m", "ragged_16", "chunk_256k",
-                             "multiblock_4x_decode_b8_128k"],
+                             "multiblock_4x_decode_b8_128k", "hybrid_swa_decode_b8_128k"],
                     help="other shapes of the pages' workloads (one GPU); the default is the "
                          "benchmark line")
     return ap.parse_args()
@@ -412,6 +412,91 @@ def run_multiblock(args, local: int, n_blocks: int = 4):
     print(json.dumps(line), flush=True)
 
 
+SWA_WINDOW = 128  # the pages give no window for the Hybrid SWA baseline: declared
+
+
+def run_hybrid_swa(args, local: int):
+    """The Hybrid SWA baseline's block on the benchmark workload, timed at the
+    kernel level beside the Hybrid Block: the same full-attention call (with
+    its scores) followed by 4 sliding-window layers (window SWA_WINDOW) instead
+    of the selection and 4 sparse layers.  Per step: 8 query tokens."""
+    import torch
+    import synth
+    from long_context_full_b200 import hs2
+    from long_context_full_b200.block import HybridBlockStep
+
+    w = synth.decode_128k(batch=BATCH, first_seq=0, context=CONTEXT)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    Q, K, V = dev(w.q), dev(w.k), dev(w.v)
+    QL = [dev(x) for x in w.q_layers]
+    step = HybridBlockStep(w.Hq, w.Hkv, w.D, torch.bfloat16, w.q_lens, w.kv_lens, w.n_layers,
+                           k=TOPK, window=WINDOW)
+    OL = [torch.empty_like(Q) for _ in range(w.n_layers)]
+
+    def swa_layers():
+        for l in range(w.n_layers):
+            hs2.hs2_swa_attn(step.problem, QL[l], K, V, SWA_WINDOW, OL[l])
+
+    for _ in range(max(3, args.warmup)):
+        step.full_attention(Q, K, V)
+        swa_layers()
+        step.select_tokens()
+        for l in range(w.n_layers):
+            step.sparse_layer(l, QL[l], K, V)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    stream = torch.cuda.current_stream()
+    Kst = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(Kst)]
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(Kst):
+        e = ev[i]
+        e[0].record(stream)
+        step.full_attention(Q, K, V)
+        e[1].record(stream)
+        swa_layers()
+        e[2].record(stream)
+        step.select_tokens()
+        e[3].record(stream)
+        for l in range(w.n_layers):
+            step.sparse_layer(l, QL[l], K, V)
+        e[4].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    ph = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in ev]).mean(axis=0)
+    t_full, t_swa, t_sel, t_sp = (float(x) for x in ph)
+    ms_step = t_full + t_swa  # the Hybrid SWA block: full attention + its SWA layers
+    value = BATCH / (ms_step * 1e-3)
+    ab = workload_accounting(w, w.n_layers)
+    hbm, hbm_kind = peaks()
+    swa_bytes = w.n_layers * (2 * BATCH * HKV * min(SWA_WINDOW, CONTEXT) * D * 2 + 2 * BATCH * HQ * D * 2)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": Kst,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V, Philox streams)",
+        "config": {"workload": f"hybrid_swa_decode_b8_128k_bf16 (window {SWA_WINDOW}, comparison)",
+                   "query_tokens_per_gpu": BATCH, "context": CONTEXT, "Hq": HQ, "Hkv": HKV, "D": D,
+                   "swa_window": SWA_WINDOW, "swa_layers": w.n_layers,
+                   "l2": f"inputs larger than L2: {ab['kv'] / 2**30:.2f} GiB of K/V per step",
+                   "parallelism": "dp1"},
+        "phase_ms": {"full_attn_scores": t_full, "swa_x4": t_swa,
+                     "hybrid_block_select": t_sel, "hybrid_block_sparse_x4": t_sp},
+        "hybrid_block_ms_per_step": t_full + t_sel + t_sp,
+        "roofline": {"kernel": "hs2_swa_attn x4 (window rows gathered)", "bound": "hbm",
+                     "achieved": swa_bytes / (t_swa * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": swa_bytes / (t_swa * 1e-3) / 1e9 / hbm, "peak_kind": hbm_kind,
+                     "traffic": None, "algorithmic_bytes": swa_bytes},
+        "gpu_launches": Kst * (3 + w.n_layers),
+        "clocks": clk,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
@@ -436,6 +521,10 @@ def main():
         if world > 1:
             raise SystemExit("--workload other than the default runs on one GPU")
         return run_multiblock(args, local)
+    if args.workload == "hybrid_swa_decode_b8_128k":
+        if world > 1:
+            raise SystemExit("--workload other than the default runs on one GPU")
+        return run_hybrid_swa(args, local)
 
     batch, context = args.batch, args.context
     if args.workload == "decode_b8_128k":

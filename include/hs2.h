@@ -181,6 +181,21 @@ hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K,
                            size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * hs2_swa_attn - the sliding-window attention layer of the Hybrid SWA baseline
+ * that the pages compare HySparse2 against ([OH] "From Hybrid SWA to
+ * HySparse2 ...": the MiMo-V2 models mixed a few full-attention layers with
+ * layers that attend only to a local neighbourhood).  For every query row at
+ * position t and query head h of KV group g:
+ *   O_h = sum_{j = max(0, t-window+1)}^{t} softmax_j(scale * q_h . k_{g,j}) v_{g,j}
+ * The pages give no window size; it is an argument (window >= 1).  Q, O
+ * [total_q, Hq, D]; K, V the layer's cache [total_kv, Hkv, D].  No workspace.
+ * It runs the sparse-attention kernels with the window in place of an index
+ * list; the result equals hs2_sparse_attn given the window positions.
+ */
+hs2_status hs2_swa_attn(const hs2_problem* p, const void* Q, const void* K, const void* V,
+                        int32_t window, void* O, void* stream);
+
+/* ---------------------------------------------------------------------------
  * hs2_kv_append - writes the K/V rows of a step's new tokens into the KV cache
  * that the full-attention layer produces and its sparse layers reuse ([HT]
  * "Two-Level KV Sharing"; [OH]: decoding extends the cache a token at a time).

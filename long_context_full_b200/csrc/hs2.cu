@@ -511,15 +511,12 @@ hs2_status hs2_sparse_attn_workspace_size(const hs2_problem* p, int32_t idx_stri
   return HS2_OK;
 }
 
-hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K, const void* V,
-                           const int32_t* idx, const int32_t* count, int32_t idx_stride, void* O_l,
-                           void* workspace, size_t workspace_bytes, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
-  hs2_status s = check_problem(p);
-  if (s != HS2_OK) return s;
-  if (!Q_l || !K || !V || !idx || !count || !O_l || idx_stride < 1) return HS2_ERR_INVALID_ARG;
-  if (!aligned16(Q_l) || !aligned16(K) || !aligned16(V) || !aligned16(O_l)) return HS2_ERR_INVALID_ARG;
+namespace {
+// One sparse-attention launch: index mode (idx/count) or window mode (window > 0).
+hs2_status run_sparse(const hs2_problem* p, const void* Q_l, const void* K, const void* V,
+                      const int32_t* idx, const int32_t* count, int32_t idx_stride, int32_t window,
+                      void* O_l, void* stream) {
+  hs2_status s;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != HS2_OK) return s;
   const int64_t rows = p->total_q * p->Hkv;
@@ -528,6 +525,7 @@ hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K,
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   SparseArgs a{};
   a.Q = Q_l; a.K = K; a.V = V; a.idx = idx; a.count = count; a.idx_stride = idx_stride;
+  a.window = window;
   a.qoff = p->q_offsets; a.kvoff = p->kv_offsets;
   a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = p->Hq / p->Hkv;
   a.total_q = p->total_q; a.total_kv = p->total_kv; a.scale = p->scale;
@@ -545,6 +543,28 @@ hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K,
     else e = launch_cluster(k_sparse_f32<16>, ctas, 32 * kSpWarps, 0, kSpCluster, st, a);
   }
   return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+}  // namespace
+
+hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K, const void* V,
+                           const int32_t* idx, const int32_t* count, int32_t idx_stride, void* O_l,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (!Q_l || !K || !V || !idx || !count || !O_l || idx_stride < 1) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q_l) || !aligned16(K) || !aligned16(V) || !aligned16(O_l)) return HS2_ERR_INVALID_ARG;
+  return run_sparse(p, Q_l, K, V, idx, count, idx_stride, 0, O_l, stream);
+}
+
+hs2_status hs2_swa_attn(const hs2_problem* p, const void* Q, const void* K, const void* V,
+                        int32_t window, void* O, void* stream) {
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (!Q || !K || !V || !O || window < 1) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return HS2_ERR_INVALID_ARG;
+  return run_sparse(p, Q, K, V, nullptr, nullptr, 0, window, O, stream);
 }
 
 // ---------------------------------------------------------------------------

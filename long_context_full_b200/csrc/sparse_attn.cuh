@@ -15,6 +15,11 @@
 // through distributed shared memory - CTA c finishing the heads h = c mod
 // kSpCluster after a single cluster barrier.  No workspace, no global round
 // trip, no atomics.
+//
+// The same kernels run the sliding-window layer of the Hybrid SWA baseline
+// ("Xiaomi Releases HySparse2, Targeting Long-Horizon Reasoning for Agents",
+// section "From Hybrid SWA to HySparse2, ..."): window mode replaces the index
+// list by the contiguous positions max(0, t-window+1) .. t.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -35,9 +40,10 @@ struct SparseArgs {
   const void* Q;        // [total_q, Hq, D], this layer's queries
   const void* K;        // [total_kv, Hkv, D]
   const void* V;
-  const int32_t* idx;   // [rows, idx_stride]
-  const int32_t* count; // [rows]
+  const int32_t* idx;   // [rows, idx_stride] (index mode)
+  const int32_t* count; // [rows] (index mode)
   int idx_stride;
+  int window;           // > 0: window mode, positions max(0, t-window+1) .. t, no index list
   const int64_t* qoff;
   const int64_t* kvoff;
   int B, Hq, Hkv, G;
@@ -60,10 +66,15 @@ __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int c
   const QueryRow q = query_row(a.qoff, a.kvoff, a.B, s.qi);
   s.kv_start = q.kv_start;
   s.t = q.t;
-  int cnt = __ldg(a.count + s.r);
-  if (cnt < 0 || cnt > a.idx_stride) {
-    if (threadIdx.x == 0 && rank == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
-    cnt = cnt < 0 ? 0 : a.idx_stride;
+  int cnt;
+  if (a.window > 0) {  // sliding window: the last min(window, t + 1) positions
+    cnt = (int)(s.t + 1 < 0 ? 0 : (s.t + 1 < a.window ? s.t + 1 : a.window));
+  } else {
+    cnt = __ldg(a.count + s.r);
+    if (cnt < 0 || cnt > a.idx_stride) {
+      if (threadIdx.x == 0 && rank == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+      cnt = cnt < 0 ? 0 : a.idx_stride;
+    }
   }
   s.cnt = cnt;
   int per = (cnt + cs - 1) / cs;
@@ -73,11 +84,11 @@ __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int c
   return s;
 }
 
-// Cache position of list entry i of the CTA's share, or -1 (recorded) if
-// outside 0..t.
+// Cache position of list entry i of the CTA's share (window mode: the i-th
+// position of the window), or -1 (recorded) if outside 0..t.
 __device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& s, int i,
                                               bool record) {
-  const int64_t pos = __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
+  const int64_t pos = a.window > 0 ? s.t - s.cnt + 1 + s.j0 + i : __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
   if (pos < 0 || pos > s.t || s.kv_start + pos >= a.total_kv) {
     if (record) record_error(a.err, HS2_ERR_DEVICE_INPUT);
     return -1;
