@@ -90,7 +90,9 @@ hs2_status device_info(DeviceInfo** out) {
                              dec_smem) != cudaSuccess)
       return HS2_ERR_CUDA;
     if (cudaFuncSetAttribute(k_sparse_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSpSmem) != cudaSuccess)
+                             (int)kSpSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(k_sparse_rows_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSrSmem) != cudaSuccess)
       return HS2_ERR_CUDA;
     if (set_chunk_tc_smem<1>() != cudaSuccess || set_chunk_tc_smem<2>() != cudaSuccess ||
         set_chunk_tc_smem<4>() != cudaSuccess || set_chunk_tc_smem<8>() != cudaSuccess)
@@ -532,7 +534,10 @@ hs2_status run_sparse(const hs2_problem* p, const void* Q_l, const void* K, cons
   a.O = O_l; a.err = dev->err;
   const unsigned ctas = (unsigned)(rows * kSpCluster);
   cudaError_t e;
-  if (p->dtype == HS2_BF16) {
+  if (p->dtype == HS2_BF16 && rows >= 4 * (int64_t)dev->sms) {
+    // many rows (a chunk of queries): one CTA per row, no cluster
+    e = launch(k_sparse_rows_bf16, dim3((unsigned)rows), dim3(32 * kSrWarps), kSrSmem, st, 0, a);
+  } else if (p->dtype == HS2_BF16) {
     e = launch_cluster(k_sparse_bf16, ctas, 32 * kSpWarps, kSpSmem, kSpCluster, st, a);
   } else {
     const int G = a.G;

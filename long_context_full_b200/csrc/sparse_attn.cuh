@@ -291,6 +291,177 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
 }
 
 // ----------------------------------------------------------------------------
+// bf16, one CTA per (query, KV group) row, for launches with many rows (a
+// chunk of queries): no cluster.  Each of the kSrWarps warps streams its own
+// 16-key slices of the row's list (slices w, w + kSrWarps, ...) through a
+// private two-deep shared-memory ring with cp.async (the copy of its next
+// slice overlaps the tensor-core work on this one), keeps its own online
+// softmax, and the warps merge once at the end.  No CTA-wide barrier in the
+// main loop.
+// ----------------------------------------------------------------------------
+constexpr int kSrWarps = 4;
+constexpr int kSrSlice = 16 * kSpRowBytes;             // 16 rows of K (or V), padded
+constexpr size_t kSrSmem = (size_t)kSrWarps * 2 * 2 * kSrSlice;  // warps x ring x (K, V)
+
+__global__ void __launch_bounds__(32 * kSrWarps) k_sparse_rows_bf16(const __grid_constant__ SparseArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
+  extern __shared__ __align__(128) uint8_t sr_smem[];
+  __shared__ float wm[kSrWarps * 8], wl[kSrWarps * 8];
+  const SpRow s = sparse_row(a, 0, 1);  // the whole row (one CTA, rank 0 of 1)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bf16* K = static_cast<const bf16*>(a.K);
+  const bf16* V = static_cast<const bf16*>(a.V);
+  uint8_t* ring = sr_smem + (size_t)warp * 2 * 2 * kSrSlice;  // [buffer][K, V][16 rows]
+
+  const int r = lane >> 2, qd = lane & 3;
+  const int h0 = 2 * qd, h1 = 2 * qd + 1;
+  const float NEG = -INFINITY;
+  const bf16* Q = static_cast<const bf16*>(a.Q);
+  uint32_t qf[8][2];
+  const bf16* qrow = Q + ((s.qi * a.Hq) + (int64_t)s.g * a.G + r) * kD;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    if (r < a.G) {
+      qf[kk][0] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * qd);
+      qf[kk][1] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * qd);
+    } else {
+      qf[kk][0] = qf[kk][1] = 0u;
+    }
+  }
+  float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
+  float o[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+
+  const int nslices = (s.n + 15) / 16;
+  // issue the gather of slice sl into ring buffer buf: lane l copies 16-byte
+  // piece l (K: l < 16, V: l >= 16) of each of the slice's 16 rows; returns the
+  // slice's positions (lane i < 16: row i's, -1 when invalid or past the list)
+  auto gather = [&](int sl, int buf) -> int64_t {
+    const int i = lane & 15;
+    const int64_t mypos = (sl * 16 + i < s.n) ? sparse_pos(a, s, sl * 16 + i, lane < 16) : -1;
+    uint8_t* dK = ring + (size_t)buf * 2 * kSrSlice;
+    uint8_t* dV = dK + kSrSlice;
+    const int c16 = lane & 15;
+    const bf16* base = lane < 16 ? K : V;
+    uint8_t* dst0 = lane < 16 ? dK : dV;
+#pragma unroll
+    for (int row = 0; row < 16; ++row) {
+      const int64_t pos = __shfl_sync(0xffffffffu, mypos, row);
+      const bool ok = pos >= 0;
+      const bf16* src = ok ? base + ((s.kv_start + pos) * a.Hkv + s.g) * kD + c16 * 8 : base;
+      cp_async16(dst0 + (size_t)row * kSpRowBytes + c16 * 16, src, ok ? 16 : 0);
+    }
+    cp_async_commit();
+    return mypos;
+  };
+
+  int sl = warp;
+  int64_t pos_cur = sl < nslices ? gather(sl, 0) : -1;
+  int buf = 0;
+  for (; sl < nslices; sl += kSrWarps) {
+    const int nxt = sl + kSrWarps;
+    int64_t pos_nxt = -1;
+    if (nxt < nslices) {
+      pos_nxt = gather(nxt, buf ^ 1);
+      cp_async_wait_prev();  // this slice's copies have landed (the next may be in flight)
+    } else {
+      cp_async_wait_all_groups();
+    }
+    __syncwarp();
+    const uint32_t skb = smem_u32(ring + (size_t)buf * 2 * kSrSlice);
+    const uint32_t svb = skb + kSrSlice;
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int row = ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int chunk = kk * 2 + (lane >> 4);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(a0, a1, a2, a3, skb + row * kSpRowBytes + chunk * 16);
+        mma_bf16(c, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+      }
+    }
+    const bool vlo = __shfl_sync(0xffffffffu, pos_cur, r) >= 0;
+    const bool vhi = __shfl_sync(0xffffffffu, pos_cur, r + 8) >= 0;
+    const float x0 = vlo ? c[0] * a.scale : NEG, x1 = vlo ? c[1] * a.scale : NEG;
+    const float x2 = vhi ? c[2] * a.scale : NEG, x3 = vhi ? c[3] * a.scale : NEG;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float al0 = (mn0 == NEG) ? 1.f : exp_shift(m0, mn0);
+    const float al1 = (mn1 == NEG) ? 1.f : exp_shift(m1, mn1);
+    const float p0v = exp_shift(x0, mn0), p1v = exp_shift(x1, mn1);
+    const float p2v = exp_shift(x2, mn0), p3v = exp_shift(x3, mn1);
+    l0 = l0 * al0 + (p0v + p2v);
+    l1 = l1 * al1 + (p1v + p3v);
+    m0 = mn0;
+    m1 = mn1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      o[i][0] *= al0; o[i][1] *= al1; o[i][2] *= al0; o[i][3] *= al1;
+    }
+    const uint32_t b0 = movmatrix_t(pack_bf16(p0v, p1v));
+    const uint32_t b1 = movmatrix_t(pack_bf16(p2v, p3v));
+    {
+      const int row = ((lane >> 4) & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int chunk = mt * 2 + ((lane >> 3) & 1);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(a0, a1, a2, a3, svb + row * kSpRowBytes + chunk * 16);
+        mma_bf16(o[mt], a0, a1, a2, a3, b0, b1);
+      }
+    }
+    __syncwarp();  // the buffer is read before the gather after next overwrites it
+    pos_cur = pos_nxt;
+    buf ^= 1;
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  if (r == 0) {
+    wm[warp * 8 + h0] = m0; wl[warp * 8 + h0] = l0;
+    wm[warp * 8 + h1] = m1; wl[warp * 8 + h1] = l1;
+  }
+  // the warp's partial O goes into its own ring (its copies have all landed
+  // and been read): 8 heads x D floats = 4 KB of the warp's 17 KB
+  float* wo_mine = reinterpret_cast<float*>(ring);
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int d = mt * 16 + r;
+    wo_mine[h0 * kD + d] = o[mt][0];
+    wo_mine[h0 * kD + d + 8] = o[mt][2];
+    wo_mine[h1 * kD + d] = o[mt][1];
+    wo_mine[h1 * kD + d + 8] = o[mt][3];
+  }
+  __syncthreads();
+  auto wo = [&](int w, int h, int d) {
+    return reinterpret_cast<const float*>(sr_smem + (size_t)w * 2 * 2 * kSrSlice)[h * kD + d];
+  };
+  // merge the warps: thread (head h, dims) finishes O
+  bf16* O = static_cast<bf16*>(a.O);
+  for (int e = threadIdx.x; e < a.G * kD; e += blockDim.x) {
+    const int h = e / kD, d = e % kD;
+    float M = -INFINITY;
+    for (int w = 0; w < kSrWarps; ++w) M = fmaxf(M, wm[w * 8 + h]);
+    float L = 0.f, acc = 0.f;
+    for (int w = 0; w < kSrWarps; ++w) {
+      const float wt = exp_shift(wm[w * 8 + h], M);
+      L = fmaf(wl[w * 8 + h], wt, L);
+      acc = fmaf(wo(w, h, d), wt, acc);
+    }
+    O[(s.qi * a.Hq + (int64_t)s.g * a.G + h) * kD + d] = from_f<bf16>(L > 0.f ? acc / L : 0.f);
+  }
+}
+
+// ----------------------------------------------------------------------------
 // float32 on the CUDA cores: each warp takes every 4th index of the CTA's share
 // and reads its K/V rows directly (lane i holds dims 4i..4i+3).
 // ----------------------------------------------------------------------------
