@@ -54,7 +54,8 @@ def parse():
                     help="cached tokens per sequence (smaller only for profiling captures)")
     ap.add_argument("--workload", default="decode_b8_128k",
                     choices=["decode_b8_128k", "needle_1m", "ragged_16", "chunk_256k",
-                             "multiblock_4x_decode_b8_128k", "hybrid_swa_decode_b8_128k"],
+                             "multiblock_4x_decode_b8_128k", "hybrid_swa_decode_b8_128k",
+                             "kv_bridge_262k"],
                     help="other shapes of the pages' workloads (one GPU); the default is the "
                          "benchmark line")
     return ap.parse_args()
@@ -497,6 +498,66 @@ def run_hybrid_swa(args, local: int):
     print(json.dumps(line), flush=True)
 
 
+BRIDGE_HIDDEN = 4096  # the pages give no hidden size: declared
+
+
+def run_kv_bridge(args, local: int):
+    """KV Bridging GEMM: K and V of 264,192 cache rows (the chunk workload's
+    cache) from hidden states of width BRIDGE_HIDDEN, Hkv = 4, D = 128.
+    Tensor-bound: 2 * rows * hidden * 2 * Hkv * D flops per call."""
+    import torch
+    from long_context_full_b200 import hs2
+
+    rows, hidden, ncols = 264192, BRIDGE_HIDDEN, HKV * D
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1250)
+    H = torch.randn(rows, hidden, device="cuda", generator=g).to(torch.bfloat16)
+    Wk = (torch.randn(ncols, hidden, device="cuda", generator=g) / math.sqrt(hidden)).to(torch.bfloat16)
+    Wv = (torch.randn(ncols, hidden, device="cuda", generator=g) / math.sqrt(hidden)).to(torch.bfloat16)
+    K = torch.empty(rows, HKV, D, dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    ko = torch.tensor([0, rows], dtype=torch.int64, device="cuda")
+    qo = torch.tensor([0, 0], dtype=torch.int64, device="cuda")
+    p = hs2.make_problem(1, HQ, HKV, D, hs2.HS2_BF16, qo, ko, 0, rows, 0, rows, 0.088)
+    for _ in range(max(3, args.warmup)):
+        hs2.hs2_kv_bridge(p, H, hidden, Wk, Wv, K, V)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    stream = torch.cuda.current_stream()
+    Kst = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(stream)
+    for _ in range(Kst):
+        hs2.hs2_kv_bridge(p, H, hidden, Wk, Wv, K, V)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    ms = start.elapsed_time(end) / Kst
+    flops = 2.0 * rows * hidden * 2 * ncols
+    tf, tf_kind = tensor_peak()
+    achieved = flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "KV Bridging: cache rows built per second (K and V projections)",
+        "value": rows / (ms * 1e-3), "unit": "cache-tok/s", "n_gpus": 1, "steps": Kst,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) hidden states and weights)",
+        "config": {"workload": f"kv_bridge_262k (hidden {hidden}, declared)", "rows": rows,
+                   "hidden": hidden, "Hkv": HKV, "D": D, "parallelism": "dp1",
+                   "l2": f"inputs larger than L2: {rows * hidden * 2 / 2**30:.2f} GiB of hidden states"},
+        "roofline": {"kernel": "k_kv_bridge<256>", "bound": "tensor", "achieved": achieved,
+                     "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "peak_kind": tf_kind,
+                     "traffic": None, "algorithmic_flops": flops},
+        "gpu_launches": Kst,
+        "clocks": clk,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
@@ -521,6 +582,10 @@ def main():
         if world > 1:
             raise SystemExit("--workload other than the default runs on one GPU")
         return run_multiblock(args, local)
+    if args.workload == "kv_bridge_262k":
+        if world > 1:
+            raise SystemExit("--workload other than the default runs on one GPU")
+        return run_kv_bridge(args, local)
     if args.workload == "hybrid_swa_decode_b8_128k":
         if world > 1:
             raise SystemExit("--workload other than the default runs on one GPU")

@@ -196,6 +196,23 @@ hs2_status hs2_swa_attn(const hs2_problem* p, const void* Q, const void* K, cons
                         int32_t window, void* O, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * hs2_kv_bridge - KV Bridging ([HT] "Two-Level KV Sharing"): the KV cache of
+ * a Cross-Decoder full-attention layer computed from the hidden states of the
+ * matching Self-Decoder full-attention layer, one GEMM per matrix:
+ *   K[n, g, :] = sum_i H[n, i] Wk_t[g*D + :, i]    (K = H Wk, with Wk_t = Wk^T)
+ *   V[n, g, :] = sum_i H[n, i] Wv_t[g*D + :, i]
+ * for every cache row n < total_kv.  The pages give neither the hidden size
+ * nor the weights: both are arguments.  bf16 only (HS2_ERR_UNSUPPORTED
+ * otherwise), fp32 accumulation, outputs rounded to bf16.
+ * H [total_kv, hidden], Wk_t and Wv_t [Hkv*D, hidden] (row-major: one output
+ * column's weights contiguous); hidden a positive multiple of 64.  K, V
+ * [total_kv, Hkv, D]: written (all rows).  Only total_kv, Hkv, D and dtype of
+ * the problem are used.  No workspace.
+ */
+hs2_status hs2_kv_bridge(const hs2_problem* p, const void* H, int32_t hidden, const void* Wk_t,
+                         const void* Wv_t, void* K, void* V, void* stream);
+
+/* ---------------------------------------------------------------------------
  * hs2_kv_append - writes the K/V rows of a step's new tokens into the KV cache
  * that the full-attention layer produces and its sparse layers reuse ([HT]
  * "Two-Level KV Sharing"; [OH]: decoding extends the cache a token at a time).

@@ -13,6 +13,7 @@
 #include "decode_attn.cuh"
 #include "select.cuh"
 #include "kv_append.cuh"
+#include "bridge.cuh"
 #include "sparse_attn.cuh"
 #include "chunk_attn.cuh"
 #include "chunk_tc.cuh"
@@ -101,6 +102,11 @@ hs2_status device_info(DeviceInfo** out) {
                              kSelSmemKeys * 4) != cudaSuccess ||
         cudaFuncSetAttribute(k_select_cluster<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSelSmemKeys * 4) != cudaSuccess)
+      return HS2_ERR_CUDA;
+    if (cudaFuncSetAttribute(k_kv_bridge<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bridge_smem<256>()) != cudaSuccess ||
+        cudaFuncSetAttribute(k_kv_bridge<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bridge_smem<128>()) != cudaSuccess)
       return HS2_ERR_CUDA;
     constexpr int ss_smem = kSsCap * 8 + kSsSortMax * 4;
     if (cudaFuncSetAttribute(k_select_sampled<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -195,8 +201,7 @@ DecodePlan plan_decode(const hs2_problem* p, const DeviceInfo& dev, void* ws) {
 
 // 3-D bf16 tensor map over a [rows, heads, 128] token-major array, boxes of
 // 64 dims x box_heads x box_rows, 128-byte swizzle.
-hs2_status encode_map3(CUtensorMap* map, const void* base, int64_t rows, int heads, int box_heads,
-                       int box_rows) {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     cudaDriverEntryPointQueryResult q;
@@ -204,14 +209,37 @@ hs2_status encode_map3(CUtensorMap* map, const void* base, int64_t rows, int hea
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
             cudaSuccess ||
         q != cudaDriverEntryPointSuccess || !fn)
-      return HS2_ERR_CUDA;
+      return nullptr;
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
+  return encode;
+}
+
+hs2_status encode_map3(CUtensorMap* map, const void* base, int64_t rows, int heads, int box_heads,
+                       int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return HS2_ERR_CUDA;
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)heads, (cuuint64_t)std::max<int64_t>(rows, 1)};
   const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)heads * kD * 2};
   const cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HS2_OK : HS2_ERR_CUDA;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] array, boxes of 64 columns
+// x box_rows rows, 128-byte swizzle.
+hs2_status encode_map2(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return HS2_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)std::max<int64_t>(rows, 1)};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -668,6 +696,38 @@ hs2_status hs2_kv_append(const hs2_problem* p, const void* K_new, const void* V_
   else
     launch(k_kv_append<kD * 4>, dim3(grid), dim3(kAppendThreads), 0, st, 0, kn, vn, k, v, p->q_offsets,
            p->kv_offsets, p->B, p->Hkv, p->total_q, p->total_kv, dev->err);
+  return launch_status();
+}
+
+hs2_status hs2_kv_bridge(const hs2_problem* p, const void* H, int32_t hidden, const void* Wk_t,
+                         const void* Wv_t, void* K, void* V, void* stream) {
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (p->dtype != HS2_BF16) return HS2_ERR_UNSUPPORTED;
+  if (!H || !Wk_t || !Wv_t || !K || !V || hidden < kBrKC || hidden % kBrKC != 0) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(Wk_t) || !aligned16(Wv_t) || !aligned16(K) || !aligned16(V))
+    return HS2_ERR_INVALID_ARG;
+  if (p->total_kv == 0) return HS2_OK;
+  const int64_t mtiles = (p->total_kv + kBrRows - 1) / kBrRows;
+  if (mtiles > 65535) return HS2_ERR_UNSUPPORTED;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != HS2_OK) return s;
+  const int ncols = p->Hkv * kD;
+  const int NT = ncols % 256 == 0 ? 256 : 128;
+  CUtensorMap mh, mk, mv;
+  if (encode_map2(&mh, H, p->total_kv, hidden, kBrRows) != HS2_OK ||
+      encode_map2(&mk, Wk_t, ncols, hidden, NT) != HS2_OK ||
+      encode_map2(&mv, Wv_t, ncols, hidden, NT) != HS2_OK)
+    return HS2_ERR_CUDA;
+  BridgeArgs a{};
+  a.rows = p->total_kv; a.hidden = hidden; a.ncols = ncols;
+  a.K = static_cast<bf16*>(K); a.V = static_cast<bf16*>(V); a.err = dev->err;
+  const dim3 grid((unsigned)(2 * ncols / NT), (unsigned)mtiles);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (NT == 256)
+    launch(k_kv_bridge<256>, grid, dim3(kBrThreads), bridge_smem<256>(), st, 0, mh, mk, mv, a);
+  else
+    launch(k_kv_bridge<128>, grid, dim3(kBrThreads), bridge_smem<128>(), st, 0, mh, mk, mv, a);
   return launch_status();
 }
 

@@ -41,20 +41,25 @@ state.  Sources (page title, then section):
   Targeting Long-Horizon Reasoning for Agents", section "From Hybrid SWA to
   HySparse2, Xiaomi Continues to Refine the Attention Structure".
 
+* ``kv_bridge``            - KV Bridging: a Cross-Decoder layer's K and V from the
+  Self-Decoder's hidden states, K = H W_K, V = H W_V.  "Xiaomi Unveils
+  HySparse2 for Faster Long-Context AI", section "Two-Level KV Sharing".
+
 Every function is pinned by ``tests/test_oracle_pins.py`` (``kv_append`` by
 ``tests/test_kv_append_pins.py``, ``swa_attention_row`` by
-``tests/test_swa_pins.py``) against closed forms, invariants and brute force on
-tiny inputs.
+``tests/test_swa_pins.py``, ``kv_bridge`` by ``tests/test_bridge_pins.py``)
+against closed forms, invariants and brute force on tiny inputs.
 """
 from .attention import (full_attention_row, selection_scores, sparse_attention_row,
                         run_full_attention, run_sparse_attention)
 from .selection import topk_select, block_select, candidate_count, window_range
 from .cache import kv_append
 from .swa import swa_attention_row
+from .bridge import kv_bridge
 
 __all__ = [
     "full_attention_row", "selection_scores", "sparse_attention_row",
     "run_full_attention", "run_sparse_attention",
     "topk_select", "block_select", "candidate_count", "window_range",
-    "kv_append", "swa_attention_row",
+    "kv_append", "swa_attention_row", "kv_bridge",
 ]
