@@ -22,7 +22,8 @@
 //           O_t += P V runs with A read from tensor memory.
 // Roles: warpgroup t (warps 4t .. 4t+3) does the softmax of Q tile t, one row
 // per thread (warp w reads tensor-memory lanes 32(w%4) .. +31); warp 8 issues
-// the TMA loads (Q once; K and V through separate two-stage rings); warp 9
+// the TMA loads (Q once; K and V through separate rings of two and three
+// stages); warp 9
 // issues the MMAs from one thread.  Tensor memory (512 columns): pass A, the S
 // buffers (tile t, buffer b) at 256t + 128b; pass B, S_t/P_t at 128t and O_t
 // at 256 + 128t.  S_t of the next key tile is issued right after the
@@ -40,13 +41,14 @@ namespace hs2 {
 constexpr int kTcRows = 128;                     // rows per Q tile = tensor-memory lanes
 constexpr int kTcQTiles = 2;                     // Q tiles per CTA
 constexpr int kTcKeys = 128;                     // keys per K/V tile
-constexpr int kTcStages = 2;                     // depth of the K ring and of the V ring
+constexpr int kTcKStages = 2;                    // depth of the K ring
+constexpr int kTcVStages = 3;                    // depth of the V ring (V is needed later than K)
 constexpr int kTcTileBytes = kTcKeys * kD * 2;   // a K or V tile: two swizzled [128][64] halves
 constexpr int kTcQBytes = kTcRows * kD * 2;      // one Q tile
 constexpr int kTcThreads = 32 * 10;              // 2 softmax warpgroups, TMA warp, MMA warp
 
 constexpr size_t chunk_tc_smem() {
-  return 1024 + (size_t)kTcQTiles * kTcQBytes + 2 * (size_t)kTcStages * kTcTileBytes;
+  return 1024 + (size_t)kTcQTiles * kTcQBytes + (size_t)(kTcKStages + kTcVStages) * kTcTileBytes;
 }
 
 template <int G>
@@ -57,8 +59,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int QT1 = kTcRows / G;  // queries per Q tile
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t q_full;
-  __shared__ __align__(8) uint64_t k_full[kTcStages], k_empty[kTcStages];
-  __shared__ __align__(8) uint64_t v_full[kTcStages], v_empty[kTcStages];
+  __shared__ __align__(8) uint64_t k_full[kTcKStages], k_empty[kTcKStages];
+  __shared__ __align__(8) uint64_t v_full[kTcVStages], v_empty[kTcVStages];
   __shared__ __align__(8) uint64_t sa_full[2][2], sa_free[2][2];  // pass A: [Q tile][S buffer]
   __shared__ __align__(8) uint64_t sb_full[2], pb_full[2], o_full;  // pass B: [Q tile]
   __shared__ uint32_t tmem_base_sh;
@@ -68,7 +70,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
   uint8_t* sK = base + kTcQTiles * kTcQBytes;
-  uint8_t* sV = sK + kTcStages * kTcTileBytes;
+  uint8_t* sV = sK + kTcKStages * kTcTileBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
   const int64_t nkeys = c.t0 + c.nq;  // keys [0, t_last] are visible to some row
@@ -76,9 +78,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < kTcKStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kTcVStages; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
@@ -111,42 +115,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_load_3d(sQ + t * kTcQBytes, &tmQ, &q_full, 0, g * G, (int)(c.q0 + t * QT1));
         tma_load_3d(sQ + t * kTcQBytes + kTcQBytes / 2, &tmQ, &q_full, 64, g * G, (int)(c.q0 + t * QT1));
       }
+      const uint64_t keep = policy_evict_last();
       // K fills 0 .. 2n-1 (pass A tiles, then pass B tiles); V fills 0 .. n-1
-      auto fill = [&](uint64_t* full, uint64_t* empty, uint8_t* ring, const CUtensorMap* map, int f,
-                      int j) -> bool {
-        const int st = f % kTcStages;
-        if (!mbar_wait(&empty[st], ((uint32_t)(f / kTcStages) & 1u) ^ 1u)) return false;
+      auto fill = [&](uint64_t* full, uint64_t* empty, uint8_t* ring, int nst, const CUtensorMap* map,
+                      int f, int j) -> bool {
+        const int st = f % nst;
+        if (!mbar_wait(&empty[st], ((uint32_t)(f / nst) & 1u) ^ 1u)) return false;
         const int key = (int)(c.kv0 + (int64_t)j * kTcKeys);
         uint8_t* dst = ring + st * kTcTileBytes;
         mbar_arrive_expect_tx(&full[st], kTcTileBytes);
-        tma_load_3d(dst, map, &full[st], 0, g, key);
-        tma_load_3d(dst + kTcTileBytes / 2, map, &full[st], 64, g, key);
+        // every CTA of the KV group reads this tile, twice for K: keep it in L2
+        tma_load_3d_hint(dst, map, &full[st], 0, g, key, keep);
+        tma_load_3d_hint(dst + kTcTileBytes / 2, map, &full[st], 64, g, key, keep);
         return true;
       };
       int kf = 0, vf = 0;
       for (int j = 0; j < n && ok; ++j) {
-        if ((ok = fill(k_full, k_empty, sK, &tmK, kf, j))) ++kf;
+        if ((ok = fill(k_full, k_empty, sK, kTcKStages, &tmK, kf, j))) ++kf;
       }
       for (int j = 0; j < n && ok; ++j) {
-        if (!(ok = fill(k_full, k_empty, sK, &tmK, kf, j))) break;
+        if (!(ok = fill(k_full, k_empty, sK, kTcKStages, &tmK, kf, j))) break;
         ++kf;
-        if (!(ok = fill(v_full, v_empty, sV, &tmV, vf, j))) break;
+        if (!(ok = fill(v_full, v_empty, sV, kTcVStages, &tmV, vf, j))) break;
         ++vf;
       }
       if (!ok) record_error(a.err, HS2_ERR_TIMEOUT);
       // before the CTA exits: every fill issued here has landed, and every
       // release of a stage (an MMA commit) has arrived
       if (!mbar_wait(&q_full, 0)) record_error(a.err, HS2_ERR_TIMEOUT);
-      auto drain = [&](uint64_t* full, uint64_t* empty, int nf) {
-        for (int f = nf - kTcStages; f < nf; ++f) {
+      auto drain = [&](uint64_t* full, uint64_t* empty, int nst, int nf) {
+        for (int f = nf - nst; f < nf; ++f) {
           if (f < 0) continue;
-          const uint32_t ph = (uint32_t)(f / kTcStages) & 1u;
-          if (!mbar_wait(&full[f % kTcStages], ph)) record_error(a.err, HS2_ERR_TIMEOUT);
-          if (ok && !mbar_wait(&empty[f % kTcStages], ph)) record_error(a.err, HS2_ERR_TIMEOUT);
+          const uint32_t ph = (uint32_t)(f / nst) & 1u;
+          if (!mbar_wait(&full[f % nst], ph)) record_error(a.err, HS2_ERR_TIMEOUT);
+          if (ok && !mbar_wait(&empty[f % nst], ph)) record_error(a.err, HS2_ERR_TIMEOUT);
         }
       };
-      drain(k_full, k_empty, kf);
-      drain(v_full, v_empty, vf);
+      drain(k_full, k_empty, kTcKStages, kf);
+      drain(v_full, v_empty, kTcVStages, vf);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                   idesc_s, kk > 0);
         }
       };
-      auto kwait = [&](int f) { return mbar_wait(&k_full[f % kTcStages], (uint32_t)(f / kTcStages) & 1u); };
+      auto kwait = [&](int f) { return mbar_wait(&k_full[f % kTcKStages], (uint32_t)(f / kTcKStages) & 1u); };
       // ---- pass A
       for (int j = 0; j < n && ok; ++j) {
         if (!(ok = kwait(j))) break;
@@ -175,10 +181,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = mbar_wait(&sa_free[t][b], ((uint32_t)(j >> 1) & 1u) ^ 1u))) break;
           tc_fence_after();
-          mma_s(256 * t + 128 * b, t, j % kTcStages);
+          mma_s(256 * t + 128 * b, t, j % kTcKStages);
           umma_commit(&sa_full[t][b]);
         }
-        umma_commit(&k_empty[j % kTcStages]);
+        umma_commit(&k_empty[j % kTcKStages]);
       }
       // every S buffer of pass A has been read before pass B reuses the columns
       for (int j = (n > 2 ? n - 2 : 0); j < n && ok; ++j)
@@ -187,15 +193,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // ---- pass B
       if (ok && n > 0 && (ok = kwait(n))) {
         tc_fence_after();
-        mma_s(0, 0, n % kTcStages);
+        mma_s(0, 0, n % kTcKStages);
         umma_commit(&sb_full[0]);
-        mma_s(128, 1, n % kTcStages);
+        mma_s(128, 1, n % kTcKStages);
         umma_commit(&sb_full[1]);
-        umma_commit(&k_empty[n % kTcStages]);
+        umma_commit(&k_empty[n % kTcKStages]);
       }
       for (int j = 0; j < n && ok; ++j) {
-        const int vst = j % kTcStages;
-        if (!(ok = mbar_wait(&v_full[vst], (uint32_t)(j / kTcStages) & 1u))) break;
+        const int vst = j % kTcVStages;
+        if (!(ok = mbar_wait(&v_full[vst], (uint32_t)(j / kTcVStages) & 1u))) break;
         const uint32_t vb = smem_u32(sV + vst * kTcTileBytes);
         const int kf = n + j + 1;  // the K fill of key tile j + 1
         for (int t = 0; t < 2 && ok; ++t) {
@@ -212,9 +218,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // read: tcgen05.mma from one thread execute in issue order
             if (t == 0 && !(ok = kwait(kf))) break;
             tc_fence_after();
-            mma_s(128 * t, t, kf % kTcStages);
+            mma_s(128 * t, t, kf % kTcKStages);
             umma_commit(&sb_full[t]);
-            if (t == 1) umma_commit(&k_empty[kf % kTcStages]);
+            if (t == 1) umma_commit(&k_empty[kf % kTcKStages]);
           }
         }
       }
@@ -362,9 +368,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int64_t ks = k0 + 64 * hh + 32 * cc + off;
             if (full && v4) {
               float4* dst = reinterpret_cast<float4*>(srow + ks);
+              // scores are read once, later, by the selection: stream them past L2
 #pragma unroll
               for (int i = 0; i < 32 / G / 4; ++i)
-                dst[i] = make_float4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]);
+                __stcs(dst + i, make_float4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]));
             } else if (rv) {
 #pragma unroll
               for (int i = 0; i < 32 / G; ++i)
