@@ -163,14 +163,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       const uint32_t qa0 = smem_u32(sQ);
       // S (128 x 128) = Q_t K^T into tensor columns d_col
+      // base descriptors once; per 16-wide k step only the start address moves
+      const uint64_t qd[2] = {umma_desc_sw128(qa0, 16, 1024), umma_desc_sw128(qa0 + kTcQBytes, 16, 1024)};
+      const uint64_t kd0 = umma_desc_sw128(smem_u32(sK), 16, 1024);
       auto mma_s = [&](uint32_t d_col, int t, int kst) {
-        const uint32_t qa = qa0 + t * kTcQBytes;
-        const uint32_t kb = smem_u32(sK + kst * kTcTileBytes);
+        const uint64_t kd = umma_desc_add(kd0, kst * kTcTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kTcTileBytes / 2) + (kk & 3) * 32;
-          umma_ss(tmem + d_col, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
-                  idesc_s, kk > 0);
+          umma_ss(tmem + d_col, umma_desc_add(qd[t], off), umma_desc_add(kd, off), idesc_s, kk > 0);
         }
       };
       auto kwait = [&](int f) { return mbar_wait(&k_full[f % kTcKStages], (uint32_t)(f / kTcKStages) & 1u); };
@@ -202,15 +203,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int j = 0; j < n && ok; ++j) {
         const int vst = j % kTcVStages;
         if (!(ok = mbar_wait(&v_full[vst], (uint32_t)(j / kTcVStages) & 1u))) break;
-        const uint32_t vb = smem_u32(sV + vst * kTcTileBytes);
+        const uint64_t vd = umma_desc_sw128(smem_u32(sV + vst * kTcTileBytes), kTcTileBytes / 2, 1024);
         const int kf = n + j + 1;  // the K fill of key tile j + 1
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = mbar_wait(&pb_full[t], (uint32_t)j & 1u))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTcKeys / 16; ++kk)
-            umma_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8,
-                    umma_desc_sw128(vb + kk * 2048, kTcTileBytes / 2, 1024), idesc_o,
+            umma_ts(tmem + 256 + 128 * t, tmem + 128 * t + kk * 8, umma_desc_add(vd, kk * 2048), idesc_o,
                     (j > 0 || kk > 0) ? 1u : 0u);
           if (t == 1) umma_commit(&v_empty[vst]);
           if (j + 1 < n) {
