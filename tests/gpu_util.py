@@ -10,7 +10,12 @@ import synth
 from long_context_full_b200 import hs2
 from long_context_full_b200.block import HybridBlockStep
 
-# Tolerances (stated by the target):
+# Tolerances.  bf16 and fp32 outputs: the stated bounds (fp32 made row-relative,
+# because element-wise relative error is unbounded near zero).  Scores: from the
+# fp32 arithmetic - logits are fp32 sums of 128 exact bf16 products (~1e-7),
+# exponentials within 2 ulp, row sums split into independent partials, at most
+# G rounded terms per score - about 2e-6, with a 10x margin.  Index sets: the
+# stated near-tie rule.
 BF16_O_ABS = 2e-2        # bf16 I/O, fp32 accumulation: max |dO| per element
 F32_O_REL = 1e-5         # fp32 build: max |dO| / max |O_ref| per (query, head) row
 SCORE_REL = 2e-5         # selection scores: |ds| <= SCORE_REL * s_ref (+ tiny absolute floor)
