@@ -263,6 +263,26 @@ hs2_status hs2_block_select_noalloc(const hs2_problem* p, const float* scores,
  */
 hs2_status hs2_get_last_device_error(void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Failure-detection self-test.  The pages have no counterpart: this call
+ * exists so that a test can watch one of the library's bounded device waits
+ * run out without faulting or hanging the GPU.  It launches one 32-thread
+ * block on ``stream`` whose single waiting thread waits for an event that
+ * nothing ever produces:
+ *   - mode 0: phase 0 of a shared-memory mbarrier that expects one arrival
+ *     and never gets it (the form of every pipeline wait in the kernels);
+ *   - mode 1: a device word that no code writes (the form of a flag wait).
+ * The wait gives up after ``limit_cycles`` SM clock cycles (values above the
+ * library's own wait limit, about 4e9 cycles, are clamped to it) and records
+ * HS2_ERR_TIMEOUT in the device error word, which hs2_get_last_device_error
+ * then returns and clears.  The context stays usable.
+ *   - Returns HS2_OK once the launch is queued; HS2_ERR_INVALID_ARG for a
+ *     mode other than 0 or 1 or a negative limit (nothing launched);
+ *     HS2_ERR_CUDA if the launch fails.
+ *   - Reads and writes no caller memory.
+ */
+hs2_status hs2_wait_selftest(int32_t mode, int64_t limit_cycles, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* hs2_status_string(hs2_status s);
 

@@ -17,6 +17,7 @@
 #include "sparse_attn.cuh"
 #include "chunk_attn.cuh"
 #include "chunk_tc.cuh"
+#include "wait_selftest.cuh"
 
 namespace hs2 {
 
@@ -671,6 +672,18 @@ const char* hs2_status_string(hs2_status s) {
     case HS2_ERR_DEVICE_INPUT: return "device found inputs that break the contract";
   }
   return "unknown status";
+}
+
+hs2_status hs2_wait_selftest(int32_t mode, int64_t limit_cycles, void* stream) {
+  if (mode != 0 && mode != 1) return HS2_ERR_INVALID_ARG;
+  if (limit_cycles < 0) return HS2_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  hs2_status s = device_info(&dev);
+  if (s != HS2_OK) return s;
+  const long long limit = limit_cycles < kWaitLimitCycles ? (long long)limit_cycles : kWaitLimitCycles;
+  launch(k_wait_selftest, dim3(1), dim3(32), 0, static_cast<cudaStream_t>(stream), 0, (int)mode, limit,
+         dev->err);
+  return launch_status();
 }
 
 hs2_status hs2_kv_append(const hs2_problem* p, const void* K_new, const void* V_new, void* K,

@@ -33,7 +33,7 @@ EXPORTED = [
     "hs2_topk_workspace_size", "hs2_topk_select",
     "hs2_block_select_workspace_size", "hs2_block_select", "hs2_block_select_noalloc",
     "hs2_sparse_attn_workspace_size", "hs2_sparse_attn", "hs2_kv_append", "hs2_swa_attn",
-    "hs2_kv_bridge",
+    "hs2_kv_bridge", "hs2_wait_selftest",
     "hs2_get_last_device_error", "hs2_status_string", "hs2_version",
 ]
 
@@ -84,6 +84,7 @@ def load() -> ctypes.CDLL:
         "hs2_kv_append": [P, vp, vp, vp, vp, vp],
         "hs2_swa_attn": [P, vp, vp, vp, i32, vp, vp],
         "hs2_kv_bridge": [P, vp, i32, vp, vp, vp, vp, vp],
+        "hs2_wait_selftest": [i32, i64, vp],
         "hs2_get_last_device_error": [vp],
         "hs2_status_string": [ctypes.c_int],
         "hs2_version": [],
@@ -235,6 +236,12 @@ def hs2_kv_bridge(p: Problem, H, hidden, Wk_t, Wv_t, K, V, stream=None):
     """K = H Wk, V = H Wv into the cache layout (Wk_t, Wv_t: [Hkv*D, hidden])."""
     _check(load().hs2_kv_bridge(ctypes.byref(p), _ptr(H), int(hidden), _ptr(Wk_t), _ptr(Wv_t),
                                 _ptr(K), _ptr(V), _stream(stream)), "hs2_kv_bridge")
+
+
+def hs2_wait_selftest(mode: int, limit_cycles: int, stream=None):
+    """Queues a bounded wait that nothing ends; it records HS2_ERR_TIMEOUT."""
+    _check(load().hs2_wait_selftest(int(mode), int(limit_cycles), _stream(stream)),
+           "hs2_wait_selftest")
 
 
 def hs2_get_last_device_error(stream=None) -> int:

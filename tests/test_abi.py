@@ -97,3 +97,10 @@ def test_workspace_sizes(lib):
     rnd = lambda b: (b + 255) // 256 * 256
     nb = (10000 + 63) // 64
     assert n.value == rnd(rows * nb * 4) + rnd(rows * 16 * 4)
+
+
+def test_wait_selftest_rejects_bad_arguments_on_the_host(lib):
+    """Checked before any CUDA call, so it runs without a GPU."""
+    assert lib.hs2_wait_selftest(2, 1000, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_wait_selftest(-1, 1000, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_wait_selftest(0, -5, None) == hs2.HS2_ERR_INVALID_ARG
