@@ -113,7 +113,9 @@ typedef struct {
  * the reading this library implements).  Scores are float32; O has ``dtype``.
  *
  * Q [total_q, Hq, D], K / V [total_kv, Hkv, D]: inputs.  O [total_q, Hq, D]:
- * output.  scores [R, score_stride] float32: output, score_stride >= max_kv_len.
+ * output.  scores [R, score_stride] float32: output, score_stride >= max_kv_len
+ * (any value; rows need not be 16-byte aligned).  Entries 0..t of a row are
+ * written; entries past t are left as they were.
  * Decode (max_q_len == 1) streams the cache once; chunks (max_q_len > 1) make a
  * second pass over K to write the scores.
  * Returns HS2_OK, or INVALID_ARG / UNSUPPORTED / WORKSPACE / CUDA.
