@@ -448,11 +448,17 @@ __global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_const
   const bool vec4 = vec && (a.G & 3) == 0;
   const uint64_t dead = policy_evict_first();  // each logit is read once
 
-  // issue the copy of one tile into buffer k (all threads)
+  // issue the copy of one tile into buffer k (all threads); a tile whose
+  // offsets disagree with the totals copies nothing and is reported
   auto load_tile = [&](int64_t tile, int k) -> bool {
     int b, nk;
     int64_t q0, kb, j0;
     if (!fin_tile(a, tile, ntile_seq, &b, &q0, &kb, &j0, &nk)) return false;
+    const int64_t N = __ldg(a.kvoff + b + 1) - kb;
+    if (q0 < 0 || q0 >= a.total_q || kb < 0 || kb + N > a.total_kv || N > stride) {
+      if (threadIdx.x == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+      return false;
+    }
     const float* src = a.logits + (kb + j0) * Hq;
     float* dst = buf[k];
     if (vec) {
@@ -481,11 +487,8 @@ __global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_const
     if (have) {
       int b, nk;
       int64_t q0, kb, j0;
-      fin_tile(a, tile, ntile_seq, &b, &q0, &kb, &j0, &nk);
-      const int64_t N = __ldg(a.kvoff + b + 1) - kb;
-      if (q0 < 0 || q0 >= a.total_q || kb < 0 || kb + N > a.total_kv || N > stride) {
-        if (threadIdx.x == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
-      } else {
+      fin_tile(a, tile, ntile_seq, &b, &q0, &kb, &j0, &nk);  // checked by load_tile
+      {
         // (m_h, 1/l_h) -> (m_h * log2 e, 1/l_h): exp(x - m) = 2^(x log2 e - m log2 e)
         for (int i = threadIdx.x; i < 2 * Hq; i += kFinKeys) {
           const float v = __ldg(ml + q0 * Hq * 2 + i);

@@ -89,7 +89,7 @@ __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int c
 __device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& s, int i,
                                               bool record) {
   const int64_t pos = a.window > 0 ? s.t - s.cnt + 1 + s.j0 + i : __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
-  if (pos < 0 || pos > s.t || s.kv_start + pos >= a.total_kv) {
+  if (pos < 0 || pos > s.t || s.kv_start + pos < 0 || s.kv_start + pos >= a.total_kv) {
     if (record) record_error(a.err, HS2_ERR_DEVICE_INPUT);
     return -1;
   }
