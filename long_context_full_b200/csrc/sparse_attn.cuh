@@ -105,46 +105,78 @@ struct SpRecv {
   float o[kSpCluster][kSpOwned][kD];
 };
 
+// One untiled bulk copy (the TMA engine, no tensor map) of ``bytes`` from
+// global memory into this CTA's shared memory, completion counted on ``bar``.
+// Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load_row(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Cluster merge.  Each CTA folds its warps' partials (wm/wl [kSpWarps][GMAX],
 // wo [kSpWarps][GMAX][D]) into one partial per head and pushes it into the
 // shared memory of CTA h % cs (distributed shared memory stores); one cluster
 // barrier makes them visible, and each CTA finishes its own heads from local
 // memory.  Nothing is read remotely after the barrier, so it is the only one.
-// D threads.
+// The softmax weights exp(m_i - M) are computed once each (thread h for head
+// h's warps, thread c for source CTA c) and shared, so every thread then only
+// sums its own dimension d.  D threads.
 template <typename OT, int GMAX>
 __device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_t qi, int g,
                                                      cg::cluster_group& cl, int rank, int cs,
                                                      const float* wm, const float* wl,
                                                      const float* wo, SpRecv& recv) {
+  __shared__ float wt[kSpWarps * GMAX];        // warp weights per head
+  __shared__ float hm[GMAX], hl[GMAX];         // this CTA's (M, L) per head
+  __shared__ float ct[kSpOwned][kSpCluster];   // source-CTA weights per owned head
   const int d = threadIdx.x;
-  for (int h = 0; h < a.G; ++h) {
+  if (d < a.G) {
+    const int h = d;
     float M = -INFINITY;
     for (int w = 0; w < kSpWarps; ++w) M = fmaxf(M, wm[w * GMAX + h]);
-    float L = 0.f, acc = 0.f;
+    float L = 0.f;
     for (int w = 0; w < kSpWarps; ++w) {
-      const float wt = exp_shift(wm[w * GMAX + h], M);
-      L = fmaf(wl[w * GMAX + h], wt, L);
-      acc = fmaf(wo[(w * GMAX + h) * kD + d], wt, acc);
+      const float e = exp_shift(wm[w * GMAX + h], M);
+      wt[w * GMAX + h] = e;
+      L = fmaf(wl[w * GMAX + h], e, L);
     }
+    hm[h] = M;
+    hl[h] = L;
+  }
+  __syncthreads();
+  for (int h = 0; h < a.G; ++h) {
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSpWarps; ++w) acc = fmaf(wo[(w * GMAX + h) * kD + d], wt[w * GMAX + h], acc);
     SpRecv* dst = cl.map_shared_rank(&recv, h % cs);
     const int slot = h / cs;
     dst->o[rank][slot][d] = acc;
     if (d == 0) {
-      dst->m[rank][slot] = M;
-      dst->l[rank][slot] = L;
+      dst->m[rank][slot] = hm[h];
+      dst->l[rank][slot] = hl[h];
     }
   }
   cl.sync();
+  // owned heads h = rank, rank + cs, ...: slot (h - rank) / cs
+  const int nown = a.G > rank ? (a.G - rank + cs - 1) / cs : 0;
+  if (d < nown * cs) {
+    const int slot = d / cs, c = d % cs;
+    float M = -INFINITY;
+    for (int c2 = 0; c2 < cs; ++c2) M = fmaxf(M, recv.m[c2][slot]);
+    ct[slot][c] = exp_shift(recv.m[c][slot], M);
+  }
+  __syncthreads();
   OT* O = static_cast<OT*>(a.O);
   for (int h = rank; h < a.G; h += cs) {
     const int slot = h / cs;
-    float M = -INFINITY;
-    for (int c = 0; c < cs; ++c) M = fmaxf(M, recv.m[c][slot]);
     float L = 0.f, acc = 0.f;
     for (int c = 0; c < cs; ++c) {
-      const float wt = exp_shift(recv.m[c][slot], M);
-      L = fmaf(recv.l[c][slot], wt, L);
-      acc = fmaf(recv.o[c][slot][d], wt, acc);
+      const float e = ct[slot][c];
+      L = fmaf(recv.l[c][slot], e, L);
+      acc = fmaf(recv.o[c][slot][d], e, acc);
     }
     O[(qi * a.Hq + (int64_t)g * a.G + h) * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
   }
@@ -160,8 +192,14 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
   __shared__ float wm[kSpWarps * 8], wl[kSpWarps * 8];
   __shared__ float wo[kSpWarps * 8 * kD];
   __shared__ SpRecv recv;
+  __shared__ __align__(8) uint64_t gbar[2];  // one per copy group, one phase per piece
   cg::cluster_group cl = cg::this_cluster();
   const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  if (threadIdx.x == 0) {
+    mbar_init(&gbar[0], blockDim.x);  // every thread arrives with the bytes it copies
+    mbar_init(&gbar[1], blockDim.x);
+    fence_mbar_init();
+  }
   const SpRow s = sparse_row(a, rank, cs);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* sK = sp_smem;
@@ -191,35 +229,50 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
   for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   const uint32_t skb = smem_u32(sK), svb = smem_u32(sV);
 
-  for (int p0 = 0; p0 < s.n; p0 += kSpPiece) {
+  for (int p0 = 0, piece = 0; p0 < s.n; p0 += kSpPiece, ++piece) {
     const int pn = s.n - p0 < kSpPiece ? s.n - p0 : kSpPiece;
     const int ntile = (pn + 15) / 16;
     // the piece's cache rows (-1: past the list or invalid), read once
     for (int row = threadIdx.x; row < ntile * 16; row += blockDim.x)
       spos[row] = row < pn ? sparse_pos(a, s, p0 + row, true) : -1;
     __syncthreads();
-    // gather: 16-byte cp.async per (row, chunk), 16 chunks of K and 16 of V per
-    // row; rows past pn or with an invalid index are zero-filled (no read).  Two
-    // copy groups: the first half of the slices is scored while the second
-    // half is still in flight.
+    // gather: one bulk copy per 256-byte K row and per V row (the TMA engine
+    // moves them, no per-16-byte requests); rows past pn or with an invalid
+    // index are zero-filled by plain stores.  Two copy groups on their own
+    // barriers: the first half of the slices is scored while the second half
+    // is still in flight.  Every thread arrives once per group with the bytes
+    // of its own copies, and no copy is issued before all have arrived.
     const int nA = (ntile + 1) / 2;
     for (int grp = 0; grp < 2; ++grp) {
-      const int lo = grp == 0 ? 0 : nA * 16 * 32, hi = grp == 0 ? nA * 16 * 32 : ntile * 16 * 32;
-      for (int i = lo + (int)threadIdx.x; i < hi; i += blockDim.x) {
-        const int row = i >> 5, ch = i & 31, c16 = ch & 15;
+      const int lo = grp == 0 ? 0 : nA * 16, hi = grp == 0 ? nA * 16 : ntile * 16;
+      uint32_t bytes = 0;
+      for (int row = lo + (int)threadIdx.x; row < hi; row += blockDim.x)
+        if (spos[row] >= 0) bytes += 2 * kD * sizeof(bf16);
+      mbar_arrive_expect_tx(&gbar[grp], bytes);
+    }
+    __syncthreads();
+    for (int grp = 0; grp < 2; ++grp) {
+      const int lo = grp == 0 ? 0 : nA * 16, hi = grp == 0 ? nA * 16 : ntile * 16;
+      for (int row = lo + (int)threadIdx.x; row < hi; row += blockDim.x) {
         const int64_t pos = spos[row];
-        const bool ok = pos >= 0;
-        const bf16* base = ch < 16 ? K : V;
-        const bf16* src = ok ? base + ((s.kv_start + pos) * a.Hkv + s.g) * kD + c16 * 8 : base;
-        uint8_t* dst = (ch < 16 ? sK : sV) + (size_t)row * kSpRowBytes + c16 * 16;
-        cp_async16(dst, src, ok ? 16 : 0);
+        uint8_t* dk = sK + (size_t)row * kSpRowBytes;
+        uint8_t* dv = sV + (size_t)row * kSpRowBytes;
+        if (pos >= 0) {
+          const int64_t off = ((s.kv_start + pos) * a.Hkv + s.g) * kD;
+          bulk_load_row(dk, K + off, kD * sizeof(bf16), &gbar[grp]);
+          bulk_load_row(dv, V + off, kD * sizeof(bf16), &gbar[grp]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < kD * (int)sizeof(bf16) / 16; ++c) {
+            reinterpret_cast<uint4*>(dk)[c] = make_uint4(0u, 0u, 0u, 0u);
+            reinterpret_cast<uint4*>(dv)[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
       }
-      cp_async_commit();
     }
     for (int half = 0; half < 2; ++half) {
-      if (half == 0) cp_async_wait_prev();
-      else cp_async_wait_all_groups();
-      __syncthreads();
+      if (!mbar_wait(&gbar[half], (uint32_t)(piece & 1))) record_error(a.err, HS2_ERR_TIMEOUT);
+      __syncthreads();  // and the zero-filled rows of other threads are visible
       for (int st = (half == 0 ? 0 : nA) + warp; st < (half == 0 ? nA : ntile); st += kSpWarps) {
         float c[4] = {0.f, 0.f, 0.f, 0.f};
         {
@@ -268,6 +321,7 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
       }
     }
     __syncthreads();  // the next piece overwrites the staged rows
+    fence_proxy_async_smem();  // ... by bulk copies after these reads and stores
   }
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
