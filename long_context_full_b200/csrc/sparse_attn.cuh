@@ -7,14 +7,19 @@
 // and selection) and "Token-Level Selection and Unified Local Access" (local and
 // global tokens come from the one shared cache, in a single sparse computation).
 //
-// One thread-block cluster of kSpCluster CTAs per (query, KV group) row: CTA c
-// takes the c-th share of the row's index list, gathers those K/V rows into
-// shared memory with 16-byte cp.async copies (rows are 256 bytes: too small for
-// efficient TMA requests), runs an online softmax per warp (tensor cores for
-// bf16), folds its warps into one partial, and the cluster merges the partials
-// through distributed shared memory - CTA c finishing the heads h = c mod
-// kSpCluster after a single cluster barrier.  No workspace, no global round
-// trip, no atomics.
+// Few rows (decode): one thread-block cluster of kSpCluster CTAs per (query,
+// KV group) row.  CTA c takes the c-th share of the row's index list and
+// reads those K/V rows - bf16: one bulk copy (the TMA engine) per 256-byte row
+// into shared memory; fp32: each warp loads its rows straight into registers,
+// 16 bytes per lane - runs an online softmax per warp (tensor cores for
+// bf16), folds its warps into one partial,
+// and the cluster merges the partials through distributed shared memory, CTA c
+// finishing the heads h = c mod kSpCluster after a single cluster barrier.  No
+// workspace, no global round trip, no atomics.
+// Many rows (a chunk of queries, bf16): one CTA per row, each warp streaming
+// its own slices through a private ring with 16-byte cp.async copies; there
+// the rows mostly come from L2, where per-lane copies keep up better than one
+// TMA request per 256-byte row.
 //
 // The same kernels run the sliding-window layer of the Hybrid SWA baseline
 // ("Xiaomi Releases HySparse2, Targeting Long-Horizon Reasoning for Agents",
