@@ -23,7 +23,6 @@ import json
 import math
 import os
 import re
-import subprocess
 import sys
 import threading
 import time

@@ -1,7 +1,6 @@
 """The benchmark's data-parallel plumbing on CPU: two gloo ranks draw disjoint
 shards of one global batch (identical to drawing the batch at once), and the
 timing reduction returns the slowest rank's time."""
-import os
 import socket
 
 import numpy as np

@@ -4,11 +4,9 @@ Outputs are checked on sampled query rows the oracle recomputes one by one;
 selection is also checked bit-exactly on the oracle's own scores."""
 import numpy as np
 import pytest
-import torch
 
 import oracle
 import synth
-from long_context_full_b200 import hs2
 from tests.gpu_util import (GpuRun, OracleRows, check_O, check_index_sets, check_scores,
                             gpu_select_on, to_f64)
 

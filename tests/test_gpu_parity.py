@@ -8,7 +8,7 @@ import oracle
 import synth
 from long_context_full_b200 import hs2
 from tests.gpu_util import (GpuRun, OracleRows, check_O, check_index_sets, check_scores,
-                            gpu_select_on, to_device, to_f64)
+                            gpu_select_on, to_f64)
 
 pytestmark = pytest.mark.gpu
 

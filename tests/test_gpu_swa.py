@@ -8,7 +8,7 @@ import torch
 import oracle
 import synth
 from long_context_full_b200 import hs2
-from tests.gpu_util import check_O, to_device, to_f64, torch_dtype
+from tests.gpu_util import check_O, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
 
