@@ -259,6 +259,77 @@ hs2_status hs2_block_select_noalloc(const hs2_problem* p, const float* scores,
                                     int32_t window, int32_t* idx, int32_t* count, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Context parallelism for decode (max_q_len == 1): the KV cache of every
+ * sequence is split by position across R ranks (one process per GPU).  Rank r
+ * holds the contiguous global positions [pos0[b], pos0[b] + n_b) of sequence
+ * b, where n_b is the sequence length in the rank's own ("local") problem;
+ * the ranks' ranges of a sequence are disjoint, cover it, and are ordered by
+ * rank.  The pages describe one device ([OH], [HT] as above); the split and
+ * these calls are this library's.  Each step computes the unsplit definition
+ * of hs2_full_attn_scores / hs2_topk_select / hs2_sparse_attn exactly, up to
+ * floating-point rounding order; between the steps the caller all-gathers the
+ * small partials (e.g. NCCL over NVLink), stacking them in rank order.
+ *
+ * Per step and rank:
+ *   1. hs2_cp_attn_partial (local problem) -> O_part, ml_part; all-gather;
+ *      hs2_cp_merge -> O and the global (m, 1/l) of every (query, head).
+ *   2. hs2_cp_scores (local problem, global ml) -> this rank's scores.
+ *   3. hs2_cp_topk_local -> (score, global position) pairs; all-gather;
+ *      hs2_cp_topk_merge (global problem) -> idx, count, identical on every
+ *      rank and equal to hs2_topk_select on the unsplit scores.
+ *   4. per sparse layer: hs2_cp_sparse_partial -> O_part, ml_part;
+ *      all-gather; hs2_cp_merge -> O_l.
+ * Partials: O_part [total_q, Hq, D] float32, each (query, head) normalised by
+ * its own softmax sum; ml_part [total_q, Hq, 2] float32 = (m, 1/l), with
+ * 1/l = 0 where the rank saw no key.  Stacked: [R, ...] in rank order.
+ * Returns as the unsplit calls; HS2_ERR_UNSUPPORTED for max_q_len > 1.
+ */
+
+/* Full-attention pass over the rank's rows: partials O_part / ml_part; the
+ * logits stay in ``workspace`` (hs2_full_attn_workspace_size bytes of the same
+ * local problem) for hs2_cp_scores, which must get the same workspace. */
+hs2_status hs2_cp_attn_partial(const hs2_problem* p, const void* Q, const void* K, const void* V,
+                               float* O_part, float* ml_part, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Merge of R stacked partials of ``rows`` (query, head) rows: O [rows, D] of
+ * ``dtype`` (HS2_BF16 or HS2_F32) and, if ml is not null, the merged (m, 1/l)
+ * [rows, 2].  M = max_r m_r, w_r = l_r exp(m_r - M), O = sum_r w_r O_r / sum_r w_r. */
+hs2_status hs2_cp_merge(int64_t rows, int32_t R, const float* O_parts, const float* ml_parts, int32_t dtype,
+                        void* O, float* ml, void* stream);
+
+/* Selection scores of the rank's own keys (local positions, as
+ * hs2_full_attn_scores writes them) from the logits kept by
+ * hs2_cp_attn_partial and the merged global ml [total_q, Hq, 2]. */
+hs2_status hs2_cp_scores(const hs2_problem* p, const float* ml, float* scores, int64_t score_stride,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* The rank's top-(k + window) keys over all its positions (window positions
+ * included: at most ``window`` of them can be), as pairs pair_score /
+ * pair_pos [rows, k + window] (float32 score, int32 global position = pos0[b]
+ * + local position; unused entries have position -1).  pos0: device [B].
+ * idx_tmp [rows, k + window] and count_tmp [rows]: scratch. */
+hs2_status hs2_cp_topk_local(const hs2_problem* p, const float* scores, int64_t score_stride, int32_t k,
+                             int32_t window, const int64_t* pos0, int32_t* idx_tmp, int32_t* count_tmp,
+                             float* pair_score, int32_t* pair_pos, void* stream);
+
+/* Global selection from R stacked pair sets [R, rows, k + window] with the
+ * GLOBAL problem (global kv offsets): positions <= t - window compete, the k
+ * best by (score desc, position asc) ascending, then the window, then -1;
+ * idx [rows, k + window], count [rows], as hs2_topk_select.  R (k + window)
+ * <= 16384 and k <= 2048, else HS2_ERR_UNSUPPORTED. */
+hs2_status hs2_cp_topk_merge(const hs2_problem* p, int32_t R, int32_t k, int32_t window, const float* pair_score,
+                             const int32_t* pair_pos, int32_t* idx, int32_t* count, void* stream);
+
+/* One sparse layer over the entries of the global list idx / count (global
+ * positions, from hs2_cp_topk_merge) that fall in the rank's rows: partials
+ * O_part / ml_part.  Entries outside the rank's rows are skipped silently
+ * (so an invalid global position is not reported here). */
+hs2_status hs2_cp_sparse_partial(const hs2_problem* p, const void* Q_l, const void* K, const void* V,
+                                 const int32_t* idx, const int32_t* count, int32_t idx_stride,
+                                 const int64_t* pos0, float* O_part, float* ml_part, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Device error word.  Synchronises ``stream``, returns the first error any
  * kernel of this library recorded on the current device since the last call
  * (HS2_OK if none) and clears it.  HS2_ERR_CUDA if the synchronisation fails.

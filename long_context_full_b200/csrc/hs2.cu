@@ -18,6 +18,7 @@
 #include "chunk_attn.cuh"
 #include "chunk_tc.cuh"
 #include "wait_selftest.cuh"
+#include "context_parallel.cuh"
 
 namespace hs2 {
 
@@ -69,6 +70,7 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[kMaxDevices];
 
+constexpr size_t kCpMergeSmem = (size_t)kCpMergeCap * 8 + (size_t)kCpPickCap * 4;
 size_t finalize_smem(int Hq) { return (2 * (size_t)kFinKeys * (Hq + 4) + 2 * (size_t)Hq) * sizeof(float); }
 std::mutex g_dev_mu;
 
@@ -124,6 +126,9 @@ hs2_status device_info(DeviceInfo** out) {
     cudaGetLastError();  // a refused non-portable size is not an error
     if (cudaFuncSetAttribute(k_finalize_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)finalize_smem(kMaxHq)) != cudaSuccess)
+      return HS2_ERR_CUDA;
+    if (cudaFuncSetAttribute(k_cp_topk_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kCpMergeSmem) != cudaSuccess)
       return HS2_ERR_CUDA;
     d.ready = true;
   }
@@ -256,9 +261,28 @@ void launch_decode_f32(dim3 grid, cudaStream_t st, const DecodeArgs& a) {
   launch(k_decode_f32<GP>, dim3(grid), dim3(32 * kDecWarps), 0, st, 0, a);
 }
 
+// Decode scores from the logits the split-context pass kept and the final
+// (m, 1/l) of every (query, head).
+hs2_status launch_finalize(const hs2_problem* p, const DeviceInfo& dev, const DecodeArgs& a,
+                           const float* ml, float* scores, int64_t stride, cudaStream_t st) {
+  if (p->max_kv_len <= 0) return HS2_OK;
+  const int ntile_seq = (int)((p->max_kv_len + kFinKeys - 1) / kFinKeys);
+  const int64_t ntiles = (int64_t)p->B * ntile_seq;
+  int per_sm = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_finalize_scores, kFinKeys, finalize_smem(p->Hq));
+  const int64_t grid = std::min<int64_t>(ntiles, (int64_t)std::max(1, per_sm) * dev.sms);
+  launch(k_finalize_scores, dim3((unsigned)grid), dim3(kFinKeys), finalize_smem(p->Hq), st, 0, a, ml, scores, stride,
+         ntile_seq);
+  return launch_status();
+}
+
+// Decode: split-context pass, combine, score finalize.  partial_ml != null:
+// context-parallel partial - O is float32, the combine writes (m, 1/l) to
+// partial_ml, and no scores are made (hs2_cp_scores makes them later from the
+// logits kept in the workspace).
 hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q, const void* K,
                       const void* V, void* O, float* scores, int64_t stride, void* ws,
-                      cudaStream_t st) {
+                      cudaStream_t st, float* partial_ml = nullptr) {
   const DecodePlan pl = plan_decode(p, dev, ws);
   DecodeArgs a{};
   a.Q = Q; a.K = K; a.V = V;
@@ -272,7 +296,10 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     if (encode_kv_map(&mk, K, p) != HS2_OK || encode_kv_map(&mv, V, p) != HS2_OK) return HS2_ERR_CUDA;
     launch(k_decode_bf16<kDecStages>, dim3(grid), dim3(32 * (kDecWarps + 1)), kDecStages * kDecStageBytes + 1024, st, 0, mk, mv, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    launch(k_decode_combine<bf16>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<bf16*>(O), pl.ml);
+    if (partial_ml)
+      launch(k_decode_combine<float>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<float*>(O), partial_ml);
+    else
+      launch(k_decode_combine<bf16>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<bf16*>(O), pl.ml);
   } else {
     const int G = a.G;
     if (G <= 1) launch_decode_f32<1>(grid, st, a);
@@ -281,20 +308,12 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     else if (G <= 8) launch_decode_f32<8>(grid, st, a);
     else launch_decode_f32<16>(grid, st, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    launch(k_decode_combine<float>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<float*>(O), pl.ml);
+    launch(k_decode_combine<float>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<float*>(O),
+           partial_ml ? partial_ml : pl.ml);
   }
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  if (p->max_kv_len > 0) {
-    const int ntile_seq = (int)((p->max_kv_len + kFinKeys - 1) / kFinKeys);
-    const int64_t ntiles = (int64_t)p->B * ntile_seq;
-    int per_sm = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_finalize_scores, kFinKeys, finalize_smem(p->Hq));
-    const int64_t grid = std::min<int64_t>(ntiles, (int64_t)std::max(1, per_sm) * dev.sms);
-    launch(k_finalize_scores, dim3((unsigned)grid), dim3(kFinKeys), finalize_smem(p->Hq), st, 0, a, pl.ml, scores, stride,
-                                                                               ntile_seq);
-    if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  }
-  return HS2_OK;
+  if (partial_ml) return HS2_OK;
+  return launch_finalize(p, dev, a, pl.ml, scores, stride, st);
 }
 
 
@@ -544,9 +563,15 @@ hs2_status hs2_sparse_attn_workspace_size(const hs2_problem* p, int32_t idx_stri
 
 namespace {
 // One sparse-attention launch: index mode (idx/count) or window mode (window > 0).
+// Context-parallel options of a sparse launch (see SparseArgs).
+struct SparseShard {
+  const int64_t* pos0;
+  float* ml_out;
+};
+
 hs2_status run_sparse(const hs2_problem* p, const void* Q_l, const void* K, const void* V,
                       const int32_t* idx, const int32_t* count, int32_t idx_stride, int32_t window,
-                      void* O_l, void* stream) {
+                      void* O_l, void* stream, const SparseShard* shard = nullptr) {
   hs2_status s;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != HS2_OK) return s;
@@ -561,9 +586,12 @@ hs2_status run_sparse(const hs2_problem* p, const void* Q_l, const void* K, cons
   a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = p->Hq / p->Hkv;
   a.total_q = p->total_q; a.total_kv = p->total_kv; a.scale = p->scale;
   a.O = O_l; a.err = dev->err;
+  if (shard) {
+    a.pos0 = shard->pos0; a.ml_out = shard->ml_out; a.o_f32 = 1;
+  }
   const unsigned ctas = (unsigned)(rows * kSpCluster);
   cudaError_t e;
-  if (p->dtype == HS2_BF16 && rows >= 4 * (int64_t)dev->sms) {
+  if (p->dtype == HS2_BF16 && rows >= 4 * (int64_t)dev->sms && !shard) {
     // many rows (a chunk of queries): one CTA per row, no cluster
     e = launch(k_sparse_rows_bf16, dim3((unsigned)rows), dim3(32 * kSrWarps), kSrSmem, st, 0, a);
   } else if (p->dtype == HS2_BF16) {
@@ -672,6 +700,118 @@ const char* hs2_status_string(hs2_status s) {
     case HS2_ERR_DEVICE_INPUT: return "device found inputs that break the contract";
   }
   return "unknown status";
+}
+
+// ---------------------------------------------------------------------------
+// Context parallelism (decode): each rank holds a position range of every
+// sequence; these calls make its partials and merge the ranks' partials.
+hs2_status hs2_cp_attn_partial(const hs2_problem* p, const void* Q, const void* K, const void* V,
+                               float* O_part, float* ml_part, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !O_part || !ml_part) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O_part)) return HS2_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != HS2_OK) return s;
+  if ((s = check_ws(workspace, workspace_bytes, plan_decode(p, *dev, nullptr).bytes)) != HS2_OK) return s;
+  return run_decode(p, *dev, Q, K, V, O_part, nullptr, 0, workspace, static_cast<cudaStream_t>(stream),
+                    ml_part);
+}
+
+hs2_status hs2_cp_scores(const hs2_problem* p, const float* ml, float* scores, int64_t score_stride,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
+  if (!ml || !scores || !aligned16(scores) || score_stride < std::max<int64_t>(1, p->max_kv_len))
+    return HS2_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != HS2_OK) return s;
+  const DecodePlan pl = plan_decode(p, *dev, workspace);
+  if ((s = check_ws(workspace, workspace_bytes, pl.bytes)) != HS2_OK) return s;
+  DecodeArgs a{};
+  a.qoff = p->q_offsets; a.kvoff = p->kv_offsets;
+  a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = p->Hq / p->Hkv; a.P = pl.P;
+  a.total_q = p->total_q; a.total_kv = p->total_kv; a.scale = p->scale;
+  a.logits = pl.logits; a.err = dev->err;
+  return launch_finalize(p, *dev, a, ml, scores, score_stride, static_cast<cudaStream_t>(stream));
+}
+
+hs2_status hs2_cp_merge(int64_t rows, int32_t R, const float* O_parts, const float* ml_parts, int32_t dtype,
+                        void* O, float* ml, void* stream) {
+  if (rows < 0 || rows >= (int64_t(1) << 31) || R < 1 || !O_parts || !ml_parts || !O)
+    return HS2_ERR_INVALID_ARG;
+  if (dtype != HS2_BF16 && dtype != HS2_F32) return HS2_ERR_INVALID_ARG;
+  if (rows == 0) return HS2_OK;
+  DeviceInfo* dev;
+  hs2_status s = device_info(&dev);
+  if (s != HS2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == HS2_BF16)
+    launch(k_cp_merge<bf16>, dim3((unsigned)rows), dim3(kD), 0, st, 0, O_parts, ml_parts, (int)R, rows,
+           static_cast<bf16*>(O), ml);
+  else
+    launch(k_cp_merge<float>, dim3((unsigned)rows), dim3(kD), 0, st, 0, O_parts, ml_parts, (int)R, rows,
+           static_cast<float*>(O), ml);
+  return launch_status();
+}
+
+hs2_status hs2_cp_topk_local(const hs2_problem* p, const float* scores, int64_t score_stride, int32_t k,
+                             int32_t window, const int64_t* pos0, int32_t* idx_tmp, int32_t* count_tmp,
+                             float* pair_score, int32_t* pair_pos, void* stream) {
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
+  if (!scores || !pos0 || !idx_tmp || !count_tmp || !pair_score || !pair_pos || k < 1 || window < 0)
+    return HS2_ERR_INVALID_ARG;
+  if ((int64_t)k + window >= (int64_t(1) << 30)) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(scores) || score_stride < std::max<int64_t>(1, p->max_kv_len)) return HS2_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != HS2_OK) return s;
+  const int kk = k + window;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the local top-(k + window) over all of the rank's positions (no window of its own)
+  if ((s = run_select(p, *dev, scores, score_stride, p->max_kv_len, kk, 0, 0, idx_tmp, kk, count_tmp, st)) !=
+      HS2_OK)
+    return s;
+  const int64_t rows = p->total_q * p->Hkv;
+  if (rows == 0) return HS2_OK;
+  launch(k_cp_pack, dim3((unsigned)rows), dim3(128), 0, st, 0, scores, score_stride, idx_tmp, count_tmp, kk,
+         p->q_offsets, p->kv_offsets, p->B, p->Hkv, pos0, pair_score, pair_pos, dev->err);
+  return launch_status();
+}
+
+hs2_status hs2_cp_topk_merge(const hs2_problem* p, int32_t R, int32_t k, int32_t window, const float* pair_score,
+                             const int32_t* pair_pos, int32_t* idx, int32_t* count, void* stream) {
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
+  if (R < 1 || k < 1 || window < 0 || !pair_score || !pair_pos || !idx || !count) return HS2_ERR_INVALID_ARG;
+  if (k > kCpPickCap || (int64_t)R * (k + window) > kCpMergeCap) return HS2_ERR_UNSUPPORTED;
+  const int64_t rows = p->total_q * p->Hkv;
+  if (rows == 0) return HS2_OK;
+  if (rows >= (int64_t(1) << 31)) return HS2_ERR_UNSUPPORTED;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != HS2_OK) return s;
+  launch(k_cp_topk_merge, dim3((unsigned)rows), dim3(kCpMergeThreads), kCpMergeSmem,
+         static_cast<cudaStream_t>(stream), 0, pair_score, pair_pos, (int)R, (int)(k + window), (int)k,
+         (int)window, p->q_offsets, p->kv_offsets, p->B, p->Hkv, rows, idx, (int)(k + window), count);
+  return launch_status();
+}
+
+hs2_status hs2_cp_sparse_partial(const hs2_problem* p, const void* Q_l, const void* K, const void* V,
+                                 const int32_t* idx, const int32_t* count, int32_t idx_stride,
+                                 const int64_t* pos0, float* O_part, float* ml_part, void* stream) {
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
+  if (!Q_l || !K || !V || !idx || !count || !pos0 || !O_part || !ml_part || idx_stride < 1)
+    return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q_l) || !aligned16(K) || !aligned16(V) || !aligned16(O_part)) return HS2_ERR_INVALID_ARG;
+  const SparseShard sh{pos0, ml_part};
+  return run_sparse(p, Q_l, K, V, idx, count, idx_stride, 0, O_part, stream, &sh);
 }
 
 hs2_status hs2_wait_selftest(int32_t mode, int64_t limit_cycles, void* stream) {

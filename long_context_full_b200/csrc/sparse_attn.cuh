@@ -56,11 +56,17 @@ struct SparseArgs {
   float scale;
   void* O;              // [total_q, Hq, D]
   int* err;
+  // context-parallel partials (all zero / null otherwise):
+  const int64_t* pos0;  // [B]: the list holds global positions; this rank's local key 0 of
+                        // sequence b is global position pos0[b]; entries outside the rank's
+                        // rows are skipped without an error
+  float* ml_out;        // [total_q, Hq, 2]: (m, 1/l) of each (query, head), 1/l = 0 if no key
+  int o_f32;            // 1: O is float32 whatever the input type
 };
 
 // This CTA's share of a row: indices [j0, j0 + n) of the row's list.
 struct SpRow {
-  int64_t r, qi, kv_start, t;
+  int64_t r, qi, kv_start, t, pos0;
   int g, cnt, j0, n;
 };
 __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int cs) {
@@ -71,6 +77,7 @@ __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int c
   const QueryRow q = query_row(a.qoff, a.kvoff, a.B, s.qi);
   s.kv_start = q.kv_start;
   s.t = q.t;
+  s.pos0 = a.pos0 ? __ldg(a.pos0 + q.b) : 0;
   int cnt;
   if (a.window > 0) {  // sliding window: the last min(window, t + 1) positions
     cnt = (int)(s.t + 1 < 0 ? 0 : (s.t + 1 < a.window ? s.t + 1 : a.window));
@@ -93,7 +100,11 @@ __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int c
 // position of the window), or -1 (recorded) if outside 0..t.
 __device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& s, int i,
                                               bool record) {
-  const int64_t pos = a.window > 0 ? s.t - s.cnt + 1 + s.j0 + i : __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
+  int64_t pos = a.window > 0 ? s.t - s.cnt + 1 + s.j0 + i : __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
+  if (a.pos0) {  // a global position: another rank's row is skipped, not an error
+    pos -= s.pos0;
+    if (pos < 0 || pos > s.t) return -1;
+  }
   if (pos < 0 || pos > s.t || s.kv_start + pos < 0 || s.kv_start + pos >= a.total_kv) {
     if (record) record_error(a.err, HS2_ERR_DEVICE_INPUT);
     return -1;
@@ -183,7 +194,14 @@ __device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_
       L = fmaf(recv.l[c][slot], e, L);
       acc = fmaf(recv.o[c][slot][d], e, acc);
     }
-    O[(qi * a.Hq + (int64_t)g * a.G + h) * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
+    const int64_t orow = qi * a.Hq + (int64_t)g * a.G + h;
+    O[orow * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
+    if (a.ml_out && d == 0) {
+      float M = -INFINITY;
+      for (int c = 0; c < cs; ++c) M = fmaxf(M, recv.m[c][slot]);
+      a.ml_out[orow * 2] = M;
+      a.ml_out[orow * 2 + 1] = L > 0.f ? 1.f / L : 0.f;
+    }
   }
 }
 
@@ -346,7 +364,8 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
     wo[(warp * 8 + h1) * kD + d + 8] = o[mt][3];
   }
   __syncthreads();
-  sparse_cluster_merge<bf16, 8>(a, s.qi, s.g, cl, rank, cs, wm, wl, wo, recv);
+  if (a.o_f32) sparse_cluster_merge<float, 8>(a, s.qi, s.g, cl, rank, cs, wm, wl, wo, recv);
+  else sparse_cluster_merge<bf16, 8>(a, s.qi, s.g, cl, rank, cs, wm, wl, wo, recv);
 }
 
 // ----------------------------------------------------------------------------

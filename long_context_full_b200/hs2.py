@@ -34,6 +34,8 @@ EXPORTED = [
     "hs2_block_select_workspace_size", "hs2_block_select", "hs2_block_select_noalloc",
     "hs2_sparse_attn_workspace_size", "hs2_sparse_attn", "hs2_kv_append", "hs2_swa_attn",
     "hs2_kv_bridge", "hs2_wait_selftest",
+    "hs2_cp_attn_partial", "hs2_cp_merge", "hs2_cp_scores", "hs2_cp_topk_local",
+    "hs2_cp_topk_merge", "hs2_cp_sparse_partial",
     "hs2_get_last_device_error", "hs2_status_string", "hs2_version",
 ]
 
@@ -85,6 +87,12 @@ def load() -> ctypes.CDLL:
         "hs2_swa_attn": [P, vp, vp, vp, i32, vp, vp],
         "hs2_kv_bridge": [P, vp, i32, vp, vp, vp, vp, vp],
         "hs2_wait_selftest": [i32, i64, vp],
+        "hs2_cp_attn_partial": [P, vp, vp, vp, vp, vp, vp, sz, vp],
+        "hs2_cp_merge": [i64, i32, vp, vp, i32, vp, vp, vp],
+        "hs2_cp_scores": [P, vp, vp, i64, vp, sz, vp],
+        "hs2_cp_topk_local": [P, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp],
+        "hs2_cp_topk_merge": [P, i32, i32, i32, vp, vp, vp, vp, vp],
+        "hs2_cp_sparse_partial": [P, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp],
         "hs2_get_last_device_error": [vp],
         "hs2_status_string": [ctypes.c_int],
         "hs2_version": [],
@@ -242,6 +250,45 @@ def hs2_wait_selftest(mode: int, limit_cycles: int, stream=None):
     """Queues a bounded wait that nothing ends; it records HS2_ERR_TIMEOUT."""
     _check(load().hs2_wait_selftest(int(mode), int(limit_cycles), _stream(stream)),
            "hs2_wait_selftest")
+
+
+def hs2_cp_attn_partial(p: Problem, Q, K, V, O_part, ml_part, workspace, stream=None):
+    ws, n = _ws(workspace)
+    _check(load().hs2_cp_attn_partial(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O_part),
+                                      _ptr(ml_part), ws, n, _stream(stream)), "hs2_cp_attn_partial")
+
+
+def hs2_cp_merge(rows: int, R: int, O_parts, ml_parts, dtype, O, ml=None, stream=None):
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    _check(load().hs2_cp_merge(int(rows), int(R), _ptr(O_parts), _ptr(ml_parts), code, _ptr(O),
+                               _ptr(ml), _stream(stream)), "hs2_cp_merge")
+
+
+def hs2_cp_scores(p: Problem, ml, scores, score_stride, workspace, stream=None):
+    ws, n = _ws(workspace)
+    _check(load().hs2_cp_scores(ctypes.byref(p), _ptr(ml), _ptr(scores), int(score_stride), ws, n,
+                                _stream(stream)), "hs2_cp_scores")
+
+
+def hs2_cp_topk_local(p: Problem, scores, score_stride, k, window, pos0, idx_tmp, count_tmp,
+                      pair_score, pair_pos, stream=None):
+    _check(load().hs2_cp_topk_local(ctypes.byref(p), _ptr(scores), int(score_stride), int(k),
+                                    int(window), _ptr(pos0), _ptr(idx_tmp), _ptr(count_tmp),
+                                    _ptr(pair_score), _ptr(pair_pos), _stream(stream)),
+           "hs2_cp_topk_local")
+
+
+def hs2_cp_topk_merge(p: Problem, R, k, window, pair_score, pair_pos, idx, count, stream=None):
+    _check(load().hs2_cp_topk_merge(ctypes.byref(p), int(R), int(k), int(window), _ptr(pair_score),
+                                    _ptr(pair_pos), _ptr(idx), _ptr(count), _stream(stream)),
+           "hs2_cp_topk_merge")
+
+
+def hs2_cp_sparse_partial(p: Problem, Q_l, K, V, idx, count, idx_stride, pos0, O_part, ml_part,
+                          stream=None):
+    _check(load().hs2_cp_sparse_partial(ctypes.byref(p), _ptr(Q_l), _ptr(K), _ptr(V), _ptr(idx),
+                                        _ptr(count), int(idx_stride), _ptr(pos0), _ptr(O_part),
+                                        _ptr(ml_part), _stream(stream)), "hs2_cp_sparse_partial")
 
 
 def hs2_get_last_device_error(stream=None) -> int:
