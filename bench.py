@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--workload", default="decode_b8_128k",
                     choices=["decode_b8_128k", "needle_1m", "ragged_16", "chunk_256k",
                              "multiblock_4x_decode_b8_128k", "hybrid_swa_decode_b8_128k",
-                             "kv_bridge_262k"],
+                             "kv_bridge_262k", "cp8_needle_1m"],
                     help="other shapes of the pages' workloads (one GPU); the default is the "
                          "benchmark line")
     return ap.parse_args()
@@ -497,6 +497,100 @@ def run_hybrid_swa(args, local: int):
     print(json.dumps(line), flush=True)
 
 
+CP_RANKS = 8
+
+
+def run_cp_rank(args, local: int):
+    """Context-parallel decode of the 1M-token needle workload split by position
+    into CP_RANKS equal ranges: all ranks run on this GPU in turn for warm-up
+    (and to fill the exchanged partials), then one rank's own work per step -
+    its full-attention partial, the merges, its scores and local top-k, the
+    merged selection and the 4 sparse partials with their merges - is timed.
+    The all-gathers between the phases are not timed (one GPU here); their
+    size per rank and step is reported."""
+    import torch
+    import synth
+    from long_context_full_b200 import hs2
+    from long_context_full_b200.context_parallel import (ContextParallelDecodeStep, LocalRanks,
+                                                         shard_offsets)
+
+    w = synth.needle_1m()
+    R, N = CP_RANKS, int(w.kv_lens[0])
+    lens = [[N // R + (1 if r < N % R else 0)] for r in range(R)]
+    pos0 = shard_offsets(lens)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    Ks = [dev(w.k[pos0[r][0]:pos0[r][0] + lens[r][0]]) for r in range(R)]
+    Vs = [dev(w.v[pos0[r][0]:pos0[r][0] + lens[r][0]]) for r in range(R)]
+    Q = dev(w.q)
+    QL = [dev(x) for x in w.q_layers]
+    steps = [ContextParallelDecodeStep(r, R, w.Hq, w.Hkv, w.D, torch.bfloat16, lens, w.n_layers,
+                                       k=TOPK, window=WINDOW, scale=w.scale) for r in range(R)]
+    ranks = LocalRanks(steps)
+    for _ in range(max(3, args.warmup)):
+        ranks.run(Q, Ks, Vs, QL)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    O_parts = torch.stack([st.O_part for st in steps])
+    ml_parts = torch.stack([st.ml_part for st in steps])
+    ps = torch.stack([st.pair_score for st in steps])
+    pp = torch.stack([st.pair_pos for st in steps])
+    st = steps[0]
+    stream = torch.cuda.current_stream()
+    Kst = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(Kst)]
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(Kst):
+        e = ev[i]
+        e[0].record(stream)
+        st.attention_partial(Q, Ks[0], Vs[0])
+        e[1].record(stream)
+        st.attention_merge(O_parts, ml_parts)
+        e[2].record(stream)
+        st.local_selection()
+        e[3].record(stream)
+        st.selection_merge(ps, pp)
+        e[4].record(stream)
+        for l in range(w.n_layers):
+            st.sparse_partial(QL[l], Ks[0], Vs[0])
+            st.sparse_merge(l, O_parts, ml_parts)
+        e[5].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    ph = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(5)] for e in ev]).mean(axis=0)
+    t_attn, t_merge, t_lsel, t_smerge, t_sparse = (float(x) for x in ph)
+    ms_step = float(ph.sum())
+    B = int(w.q_lens.sum())
+    kv_bytes = 2 * lens[0][0] * w.Hkv * w.D * 2
+    hbm, hbm_kind = peaks()
+    exch = 4 * B * w.Hq * (w.D + 2) * (2 + w.n_layers) + 8 * B * w.Hkv * (TOPK + WINDOW)
+    line = {
+        "metric": METRIC, "value": B / (ms_step * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": Kst,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V with 64 needles, Philox streams)",
+        "config": {"workload": f"cp{R}_needle_b1_1m_bf16 (rank 0 of {R} context-parallel ranks; "
+                               f"all ranks run on this one GPU, the all-gathers are not timed)",
+                   "query_tokens": B, "context": N, "keys_per_rank": lens[0][0], "Hq": w.Hq,
+                   "Hkv": w.Hkv, "D": w.D, "k": TOPK, "window": WINDOW, "reuse_layers": w.n_layers,
+                   "l2": f"inputs larger than L2: {kv_bytes / 2**20:.0f} MiB of K/V per rank-step",
+                   "parallelism": f"cp{R} (emulated)"},
+        "phase_ms": {"attn_partial": t_attn, "attn_merge": t_merge, "scores_and_local_topk": t_lsel,
+                     "topk_merge": t_smerge, "sparse_partial_and_merge_x4": t_sparse},
+        "exchange_bytes_per_rank_step": exch,
+        "roofline": {"kernel": "hs2_cp_attn_partial (decode pass + combine on the rank's keys)",
+                     "bound": "hbm", "achieved": kv_bytes / (t_attn * 1e-3) / 1e9, "peak": hbm,
+                     "unit": "GB/s", "frac": kv_bytes / (t_attn * 1e-3) / 1e9 / hbm,
+                     "peak_kind": hbm_kind, "traffic": None, "algorithmic_bytes": kv_bytes},
+        "gpu_launches": Kst * (2 + 1 + 3 + 1 + 2 * w.n_layers),
+        "clocks": clk,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 BRIDGE_HIDDEN = 4096  # the pages give no hidden size: declared
 
 
@@ -589,6 +683,10 @@ def main():
         if world > 1:
             raise SystemExit("--workload other than the default runs on one GPU")
         return run_hybrid_swa(args, local)
+    if args.workload == "cp8_needle_1m":
+        if world > 1:
+            raise SystemExit("--workload other than the default runs on one GPU")
+        return run_cp_rank(args, local)
 
     batch, context = args.batch, args.context
     if args.workload == "decode_b8_128k":

@@ -96,41 +96,101 @@ __global__ void __launch_bounds__(128) k_cp_pack(const float* scores, int64_t st
 // at positions <= t - window are candidates; the k best by (score desc,
 // position asc) are written ascending, then the window max(0, t-window+1)..t,
 // then -1 padding; count = picks + window length (as hs2_topk_select).  t from
-// the global offsets.  Grid: rows; kCpMergeThreads threads; dynamic shared
-// memory: kCpMergeCap x 8 bytes of sort keys + 2048 x 4 bytes of picks.
-constexpr int kCpMergeThreads = 1024;
+// the global offsets.  The candidates are compacted into shared memory as
+// (position << 32 | score key); a three-pass radix select (11/11/10 bits)
+// finds the k-th largest score key T and how many keys equal to T to take
+// (kr); every key > T is taken, and the kr lowest positions among the keys ==
+// T (all of them in the usual case of no ties at T; else after ordering the
+// candidates by position); the picks are then sorted by position.  Grid:
+// rows; kSelThreads threads (the block-level digit search assumes it);
+// dynamic shared memory kCpMergeCap x 8 bytes of keys + kCpPickCap x 4 bytes.
+constexpr int kCpMergeThreads = kSelThreads;
 constexpr int kCpMergeCap = 16384;  // R x kk at most (a power of two)
 constexpr int kCpPickCap = 2048;    // k at most
 
-__global__ void __launch_bounds__(kCpMergeThreads) k_cp_topk_merge(
+__global__ void __launch_bounds__(kSelThreads) k_cp_topk_merge(
     const float* pair_score, const int32_t* pair_pos, int R, int kk, int k, int window,
     const int64_t* qoff, const int64_t* kvoff, int B, int Hkv, int64_t rows, int32_t* idx,
     int out_stride, int32_t* count) {
   grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ __align__(16) uint64_t cpm_keys[];
   int32_t* picks = reinterpret_cast<int32_t*>(cpm_keys + kCpMergeCap);
-  __shared__ int nvalid;
+  __shared__ uint32_t hist[kSelBins];
+  __shared__ int scan_sh[kSelThreads / 32 + 1];
+  __shared__ int nvalid, ngt, neq, ntie;
+  __shared__ uint32_t s_digit;
+  __shared__ int s_rem;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = blockIdx.x;
   const QueryRow q = query_row(qoff, kvoff, B, row / Hkv);
   const int64_t cut = q.t - window;  // candidates: positions 0..cut
-  if (threadIdx.x == 0) nvalid = 0;
+  if (threadIdx.x == 0) {
+    nvalid = 0;
+    ngt = 0;
+    neq = 0;
+    ntie = 0;
+  }
   __syncthreads();
   const int n = R * kk;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const int r = i / kk, j = i % kk;
     const int64_t at = ((int64_t)r * rows + row) * kk + j;
     const int32_t pos = __ldg(pair_pos + at);
-    uint64_t key = ~uint64_t(0);
-    if (pos >= 0 && pos <= cut) {
-      key = ((uint64_t)(~score_key(__ldg(pair_score + at))) << 32) | (uint32_t)pos;
-      atomicAdd(&nvalid, 1);
-    }
-    cpm_keys[i] = key;
+    if (pos >= 0 && pos <= cut)
+      cpm_keys[atomicAdd(&nvalid, 1)] = ((uint64_t)(uint32_t)pos << 32) | score_key(__ldg(pair_score + at));
   }
   __syncthreads();
-  sel_sort_asc(cpm_keys, n, sel_pow2_at_least(n), ~uint64_t(0));
-  const int npick = nvalid < k ? nvalid : k;
-  for (int i = threadIdx.x; i < npick; i += blockDim.x) picks[i] = (int32_t)(uint32_t)cpm_keys[i];
+  const int nv = nvalid;
+  const int npick = nv < k ? nv : k;
+  if (nv <= k) {
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) picks[i] = (int32_t)(cpm_keys[i] >> 32);
+  } else {
+    uint32_t pre = 0;
+    int need = k;
+    for (int pass = 0; pass < 3; ++pass) {
+      for (int i = threadIdx.x; i < kSelBins; i += blockDim.x) hist[i] = 0u;
+      __syncthreads();
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const uint32_t mask = pass == 2 ? 0x3FFu : 0x7FFu;
+      const int pshift = pass == 0 ? 32 : (pass == 1 ? 21 : 10);
+      for (int base = warp * 32; base < nv; base += blockDim.x) {
+        const int i = base + lane;
+        const uint32_t u = i < nv ? (uint32_t)cpm_keys[i] : 0u;
+        const bool ok = i < nv && (pass == 0 || (u >> pshift) == pre);
+        sel_hist_add(hist, (u >> shift) & mask, ok);
+      }
+      __syncthreads();
+      sel_block_find(hist, pass == 2 ? 1024 : kSelBins, need, scan_sh, &s_digit, &s_rem);
+      pre = pass == 0 ? s_digit : ((pre << (pass == 1 ? 11 : 10)) | s_digit);
+      need = s_rem;
+    }
+    const uint32_t T = pre;
+    const int kr = need;
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+      const uint32_t u = (uint32_t)cpm_keys[i];
+      if (u > T) picks[atomicAdd(&ngt, 1)] = (int32_t)(cpm_keys[i] >> 32);
+      else if (u == T) atomicAdd(&neq, 1);
+    }
+    __syncthreads();
+    const int g = ngt;
+    if (kr == neq) {  // every key equal to T is taken
+      for (int i = threadIdx.x; i < nv; i += blockDim.x)
+        if ((uint32_t)cpm_keys[i] == T) picks[g + atomicAdd(&ntie, 1)] = (int32_t)(cpm_keys[i] >> 32);
+    } else {  // more ties than places: take the lowest positions among them
+      sel_sort_asc(cpm_keys, nv, sel_pow2_at_least(nv), ~uint64_t(0));
+      const int E = (nv + blockDim.x - 1) / blockDim.x;
+      const int lo = min(nv, (int)threadIdx.x * E), hi = min(nv, lo + E);
+      int mine = 0;
+      for (int i = lo; i < hi; ++i) mine += (uint32_t)cpm_keys[i] == T;
+      int tot;
+      int tb = block_exclusive_scan(mine, scan_sh, &tot);
+      for (int i = lo; i < hi; ++i)
+        if ((uint32_t)cpm_keys[i] == T) {
+          if (tb < kr) picks[g + tb] = (int32_t)(cpm_keys[i] >> 32);
+          ++tb;
+        }
+    }
+  }
   __syncthreads();
   sel_sort_asc(picks, npick, sel_pow2_at_least(npick), INT32_MAX);
   int32_t* out = idx + row * out_stride;
