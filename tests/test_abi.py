@@ -104,3 +104,38 @@ def test_wait_selftest_rejects_bad_arguments_on_the_host(lib):
     assert lib.hs2_wait_selftest(2, 1000, None) == hs2.HS2_ERR_INVALID_ARG
     assert lib.hs2_wait_selftest(-1, 1000, None) == hs2.HS2_ERR_INVALID_ARG
     assert lib.hs2_wait_selftest(0, -5, None) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_context_parallel_calls_reject_bad_arguments_on_the_host(lib):
+    """Checked before any CUDA call, so it runs without a GPU."""
+    P = lambda **kw: ctypes.byref(_problem(**kw))
+    # chunks are not split across ranks
+    chunk = dict(max_q_len=4, total_q=4)
+    assert lib.hs2_cp_attn_partial(P(**chunk), 0x1000, 0x1000, 0x1000, 0x2000, 0x3000, None, 0,
+                                   None) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_cp_scores(P(**chunk), 0x3000, 0x4000, 128, None, 0, None) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_cp_topk_local(P(**chunk), 0x4000, 128, 1024, 128, 0x5000, 0x6000, 0x7000, 0x8000,
+                                 0x9000, None) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_cp_sparse_partial(P(**chunk), 0x1000, 0x1000, 0x1000, 0x6000, 0x7000, 1152,
+                                     0x5000, 0x2000, 0x3000, None) == hs2.HS2_ERR_UNSUPPORTED
+    # missing buffers, bad sizes
+    assert lib.hs2_cp_attn_partial(P(), 0x1000, 0x1000, 0x1000, None, 0x3000, None, 0,
+                                   None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_cp_scores(P(), 0x3000, 0x4000, 50, None, 0, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_cp_topk_local(P(), 0x4000, 128, 1024, 128, None, 0x6000, 0x7000, 0x8000, 0x9000,
+                                 None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_cp_topk_local(P(), 0x4000, 128, 0, 128, 0x5000, 0x6000, 0x7000, 0x8000, 0x9000,
+                                 None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_cp_sparse_partial(P(), 0x1000, 0x1000, 0x1000, 0x6000, 0x7000, 1152, None,
+                                     0x2000, 0x3000, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_cp_merge(-1, 2, 0x1000, 0x2000, hs2.HS2_BF16, 0x3000, None, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_cp_merge(8, 0, 0x1000, 0x2000, hs2.HS2_BF16, 0x3000, None, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_cp_merge(8, 2, 0x1000, 0x2000, 7, 0x3000, None, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_cp_merge(0, 2, 0x1000, 0x2000, hs2.HS2_BF16, 0x3000, None, None) == hs2.HS2_OK
+    # the merged selection's shared-memory limits: k <= 2048, R (k + window) <= 16384
+    assert lib.hs2_cp_topk_merge(P(), 2, 4096, 128, 0x1000, 0x2000, 0x3000, 0x4000,
+                                 None) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_cp_topk_merge(P(), 16, 1024, 128, 0x1000, 0x2000, 0x3000, 0x4000,
+                                 None) == hs2.HS2_ERR_UNSUPPORTED
+    assert lib.hs2_cp_topk_merge(P(), 0, 1024, 128, 0x1000, 0x2000, 0x3000, 0x4000,
+                                 None) == hs2.HS2_ERR_INVALID_ARG
