@@ -127,14 +127,17 @@ class ContextParallelDecodeStep:
                          self.O_layers[l], None, stream)
 
     def run(self, Q, K, V, Q_layers, all_gather, stream=None):
-        """One step on this rank; ``all_gather(t)`` stacks the ranks' ``t``."""
-        self.attention_partial(Q, K, V, stream)
-        self.attention_merge(all_gather(self.O_part), all_gather(self.ml_part), stream)
-        self.local_selection(stream)
-        self.selection_merge(all_gather(self.pair_score), all_gather(self.pair_pos), stream)
-        for l in range(self.n_layers):
-            self.sparse_partial(Q_layers[l], K, V, stream)
-            self.sparse_merge(l, all_gather(self.O_part), all_gather(self.ml_part), stream)
+        """One step on this rank; ``all_gather(t)`` stacks the ranks' ``t``.
+        Everything, the exchange included, is ordered on ``stream`` (default:
+        the current stream)."""
+        with torch.cuda.stream(stream):
+            self.attention_partial(Q, K, V)
+            self.attention_merge(all_gather(self.O_part), all_gather(self.ml_part))
+            self.local_selection()
+            self.selection_merge(all_gather(self.pair_score), all_gather(self.pair_pos))
+            for l in range(self.n_layers):
+                self.sparse_partial(Q_layers[l], K, V)
+                self.sparse_merge(l, all_gather(self.O_part), all_gather(self.ml_part))
         return self.O, self.scores, self.idx, self.count, self.O_layers
 
 
@@ -158,23 +161,25 @@ class LocalRanks:
         self.steps = list(steps)
 
     def run(self, Q, Ks, Vs, Q_layers, stream=None):
+        """One step of every rank, ordered on ``stream`` (default: the current stream)."""
         S = self.steps
-        for r, st in enumerate(S):
-            st.attention_partial(Q, Ks[r], Vs[r], stream)
-        O_parts = torch.stack([st.O_part for st in S])
-        ml_parts = torch.stack([st.ml_part for st in S])
-        for st in S:
-            st.attention_merge(O_parts, ml_parts, stream)
-        for st in S:
-            st.local_selection(stream)
-        ps = torch.stack([st.pair_score for st in S])
-        pp = torch.stack([st.pair_pos for st in S])
-        for st in S:
-            st.selection_merge(ps, pp, stream)
-        for l in range(S[0].n_layers):
+        with torch.cuda.stream(stream):
             for r, st in enumerate(S):
-                st.sparse_partial(Q_layers[l], Ks[r], Vs[r], stream)
+                st.attention_partial(Q, Ks[r], Vs[r])
             O_parts = torch.stack([st.O_part for st in S])
             ml_parts = torch.stack([st.ml_part for st in S])
             for st in S:
-                st.sparse_merge(l, O_parts, ml_parts, stream)
+                st.attention_merge(O_parts, ml_parts)
+            for st in S:
+                st.local_selection()
+            ps = torch.stack([st.pair_score for st in S])
+            pp = torch.stack([st.pair_pos for st in S])
+            for st in S:
+                st.selection_merge(ps, pp)
+            for l in range(S[0].n_layers):
+                for r, st in enumerate(S):
+                    st.sparse_partial(Q_layers[l], Ks[r], Vs[r])
+                O_parts = torch.stack([st.O_part for st in S])
+                ml_parts = torch.stack([st.ml_part for st in S])
+                for st in S:
+                    st.sparse_merge(l, O_parts, ml_parts)
