@@ -23,7 +23,8 @@
  *                         per reuse layer, each with its own queries)
  *   hs2_block_select      (comparison path) first-generation block selection
  * and, before them in a decode step, hs2_kv_append (the new tokens' K/V rows
- * written into the cache).
+ * written into the cache).  A decode step whose cache is split by position
+ * across GPUs uses the hs2_cp_* calls instead (context parallelism, below).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -51,7 +52,8 @@
  *   same workspace must not overlap.
  * Workspace.  Query the size with the matching *_workspace_size call; pass at
  *   least that many bytes, 256-byte aligned.  Its contents on entry do not
- *   matter; on return they are unspecified.
+ *   matter; on return they are unspecified - except that hs2_cp_scores reads
+ *   the logits hs2_cp_attn_partial left in the same workspace.
  * Errors.  Arguments are checked on the host before any launch; a failed check
  *   returns an error code and launches nothing.  A CUDA launch failure returns
  *   HS2_ERR_CUDA.  Conditions only the device can see (offsets that disagree
