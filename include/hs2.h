@@ -54,6 +54,9 @@
  *   least that many bytes, 256-byte aligned.  Its contents on entry do not
  *   matter; on return they are unspecified - except that hs2_cp_scores reads
  *   the logits hs2_cp_attn_partial left in the same workspace.
+ * Empty steps.  When total_q = 0 (no query rows) a call checks the problem
+ *   and its scalar arguments, launches nothing and returns HS2_OK; its tensor
+ *   and workspace pointers are not used and may be null.
  * Errors.  Arguments are checked on the host before any launch; a failed check
  *   returns an error code and launches nothing.  A CUDA launch failure returns
  *   HS2_ERR_CUDA.  Conditions only the device can see (offsets that disagree
@@ -156,6 +159,8 @@ hs2_status hs2_topk_select(const hs2_problem* p, const float* scores, int64_t sc
  * block index first) contribute all their candidate positions, ascending,
  * followed by the window.
  * idx [R, n_blocks*block + window] int32 (-1 padded), count [R] int32.
+ * A row whose offsets give more candidates than score_stride is recorded as
+ * HS2_ERR_DEVICE_INPUT and gets count 0 and all -1.
  */
 hs2_status hs2_block_select_workspace_size(const hs2_problem* p, int32_t n_blocks,
                                            int32_t block, int32_t window, size_t* bytes);
@@ -251,8 +256,10 @@ hs2_status hs2_kv_append(const hs2_problem* p, const void* K_new, const void* V_
  *     runtime query, no allocation); make that first call before any stream
  *     capture.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents.  Nothing in it needs to start at zero: every entry a call reads
- *     was written earlier in the same call.  Calls that overlap on the GPU
+ *     contents.  Nothing in it needs to start at zero: every scratch entry
+ *     whose value reaches idx or count was written earlier in the same call
+ *     (a row the device rejects with HS2_ERR_DEVICE_INPUT gets count 0 and
+ *     all -1, whatever the array held).  Calls that overlap on the GPU
  *     (different streams, or host threads without ordering) race on it:
  *     serialise them.
  */

@@ -468,6 +468,7 @@ hs2_status hs2_full_attn_scores(const hs2_problem* p, const void* Q, const void*
                                 size_t workspace_bytes, void* stream) {
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
+  if (p->total_q == 0) return HS2_OK;  // no query rows: nothing to read or write
   if (!Q || !K || !V || !O || !scores) return HS2_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(scores))
     return HS2_ERR_INVALID_ARG;
@@ -475,7 +476,6 @@ hs2_status hs2_full_attn_scores(const hs2_problem* p, const void* Q, const void*
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != HS2_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (p->total_q == 0) return HS2_OK;
   if (p->max_q_len <= 1) {
     if ((s = check_ws(workspace, workspace_bytes, plan_decode(p, *dev, nullptr).bytes)) != HS2_OK) return s;
     return run_decode(p, *dev, Q, K, V, O, scores, score_stride, workspace, st);
@@ -499,8 +499,9 @@ hs2_status hs2_topk_select(const hs2_problem* p, const float* scores, int64_t sc
   (void)workspace_bytes;
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
-  if (!scores || !idx || !count || k < 1 || window < 1) return HS2_ERR_INVALID_ARG;
-  if ((int64_t)k + window >= (int64_t(1) << 30)) return HS2_ERR_INVALID_ARG;
+  if (k < 1 || window < 1 || (int64_t)k + window >= (int64_t(1) << 30)) return HS2_ERR_INVALID_ARG;
+  if (p->total_q == 0) return HS2_OK;  // no rows
+  if (!scores || !idx || !count) return HS2_ERR_INVALID_ARG;
   if (!aligned16(scores) || score_stride < std::max<int64_t>(1, p->max_kv_len)) return HS2_ERR_INVALID_ARG;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != HS2_OK) return s;
@@ -527,8 +528,10 @@ hs2_status hs2_block_select(const hs2_problem* p, const float* scores, int64_t s
                             int32_t* count, void* workspace, size_t workspace_bytes, void* stream) {
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
-  if (!scores || !idx || !count || n_blocks < 1 || block < 1 || window < 1) return HS2_ERR_INVALID_ARG;
+  if (n_blocks < 1 || block < 1 || window < 1) return HS2_ERR_INVALID_ARG;
   if ((int64_t)n_blocks * block + window >= (int64_t(1) << 30)) return HS2_ERR_INVALID_ARG;
+  if (p->total_q == 0) return HS2_OK;  // no rows: the workspace is not needed either
+  if (!scores || !idx || !count) return HS2_ERR_INVALID_ARG;
   if (!aligned16(scores) || score_stride < std::max<int64_t>(1, p->max_kv_len)) return HS2_ERR_INVALID_ARG;
   size_t need;
   if ((s = hs2_block_select_workspace_size(p, n_blocks, block, window, &need)) != HS2_OK) return s;
@@ -547,9 +550,9 @@ hs2_status hs2_block_select(const hs2_problem* p, const float* scores, int64_t s
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
   if ((s = run_select(p, *dev, bmax, nb, nb, n_blocks, window, block, bsel, n_blocks, nullptr, st)) != HS2_OK)
     return s;
-  launch(k_block_expand, dim3((unsigned)rows), dim3(256), 0, st, 0, bsel, n_blocks, p->q_offsets, p->kv_offsets, p->B,
-                                                 p->Hkv, block, window, idx,
-                                                 (int64_t)n_blocks * block + window, count);
+  launch(k_block_expand, dim3((unsigned)rows), dim3(256), 0, st, 0, bsel, n_blocks, p->q_offsets, p->kv_offsets,
+         p->B, p->Hkv, block, window, score_stride, nb, idx, (int64_t)n_blocks * block + window, count,
+         dev->err);
   return launch_status();
 }
 
@@ -615,7 +618,9 @@ hs2_status hs2_sparse_attn(const hs2_problem* p, const void* Q_l, const void* K,
   (void)workspace_bytes;
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
-  if (!Q_l || !K || !V || !idx || !count || !O_l || idx_stride < 1) return HS2_ERR_INVALID_ARG;
+  if (idx_stride < 1) return HS2_ERR_INVALID_ARG;
+  if (p->total_q == 0) return HS2_OK;  // no query rows
+  if (!Q_l || !K || !V || !idx || !count || !O_l) return HS2_ERR_INVALID_ARG;
   if (!aligned16(Q_l) || !aligned16(K) || !aligned16(V) || !aligned16(O_l)) return HS2_ERR_INVALID_ARG;
   return run_sparse(p, Q_l, K, V, idx, count, idx_stride, 0, O_l, stream);
 }
@@ -624,7 +629,9 @@ hs2_status hs2_swa_attn(const hs2_problem* p, const void* Q, const void* K, cons
                         int32_t window, void* O, void* stream) {
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
-  if (!Q || !K || !V || !O || window < 1) return HS2_ERR_INVALID_ARG;
+  if (window < 1) return HS2_ERR_INVALID_ARG;
+  if (p->total_q == 0) return HS2_OK;  // no query rows
+  if (!Q || !K || !V || !O) return HS2_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return HS2_ERR_INVALID_ARG;
   return run_sparse(p, Q, K, V, nullptr, nullptr, 0, window, O, stream);
 }
@@ -671,6 +678,7 @@ hs2_status hs2_block_select_noalloc(const hs2_problem* p, const float* scores, i
   hs2_status s = hs2_block_select_workspace_size(p, n_blocks, block, window, &need);
   if (s != HS2_OK) return s;
   if (need > kNoAllocScratchBytes) return HS2_ERR_WORKSPACE;  // larger than the fixed scratch
+  if (p->total_q == 0) return HS2_OK;  // no rows: nothing to look up or launch
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != HS2_OK) return s;
   return hs2_block_select(p, scores, score_stride, n_blocks, block, window, idx, count, scratch,
@@ -711,6 +719,7 @@ hs2_status hs2_cp_attn_partial(const hs2_problem* p, const void* Q, const void* 
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
   if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
+  if (p->total_q == 0) return HS2_OK;  // no query rows
   if (!Q || !K || !V || !O_part || !ml_part) return HS2_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O_part)) return HS2_ERR_INVALID_ARG;
   DeviceInfo* dev;
@@ -725,6 +734,7 @@ hs2_status hs2_cp_scores(const hs2_problem* p, const float* ml, float* scores, i
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
   if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
+  if (p->total_q == 0) return HS2_OK;  // no query rows
   if (!ml || !scores || !aligned16(scores) || score_stride < std::max<int64_t>(1, p->max_kv_len))
     return HS2_ERR_INVALID_ARG;
   DeviceInfo* dev;
@@ -764,9 +774,9 @@ hs2_status hs2_cp_topk_local(const hs2_problem* p, const float* scores, int64_t 
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
   if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
-  if (!scores || !pos0 || !idx_tmp || !count_tmp || !pair_score || !pair_pos || k < 1 || window < 0)
-    return HS2_ERR_INVALID_ARG;
-  if ((int64_t)k + window >= (int64_t(1) << 30)) return HS2_ERR_INVALID_ARG;
+  if (k < 1 || window < 0 || (int64_t)k + window >= (int64_t(1) << 30)) return HS2_ERR_INVALID_ARG;
+  if (p->total_q == 0) return HS2_OK;  // no rows
+  if (!scores || !pos0 || !idx_tmp || !count_tmp || !pair_score || !pair_pos) return HS2_ERR_INVALID_ARG;
   if (!aligned16(scores) || score_stride < std::max<int64_t>(1, p->max_kv_len)) return HS2_ERR_INVALID_ARG;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != HS2_OK) return s;
@@ -788,10 +798,11 @@ hs2_status hs2_cp_topk_merge(const hs2_problem* p, int32_t R, int32_t k, int32_t
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
   if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
-  if (R < 1 || k < 1 || window < 0 || !pair_score || !pair_pos || !idx || !count) return HS2_ERR_INVALID_ARG;
+  if (R < 1 || k < 1 || window < 0) return HS2_ERR_INVALID_ARG;
   if (k > kCpPickCap || (int64_t)R * (k + window) > kCpMergeCap) return HS2_ERR_UNSUPPORTED;
   const int64_t rows = p->total_q * p->Hkv;
-  if (rows == 0) return HS2_OK;
+  if (rows == 0) return HS2_OK;  // no rows
+  if (!pair_score || !pair_pos || !idx || !count) return HS2_ERR_INVALID_ARG;
   if (rows >= (int64_t(1) << 31)) return HS2_ERR_UNSUPPORTED;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != HS2_OK) return s;
@@ -807,8 +818,9 @@ hs2_status hs2_cp_sparse_partial(const hs2_problem* p, const void* Q_l, const vo
   hs2_status s = check_problem(p);
   if (s != HS2_OK) return s;
   if (p->max_q_len > 1) return HS2_ERR_UNSUPPORTED;
-  if (!Q_l || !K || !V || !idx || !count || !pos0 || !O_part || !ml_part || idx_stride < 1)
-    return HS2_ERR_INVALID_ARG;
+  if (idx_stride < 1) return HS2_ERR_INVALID_ARG;
+  if (p->total_q == 0) return HS2_OK;  // no query rows
+  if (!Q_l || !K || !V || !idx || !count || !pos0 || !O_part || !ml_part) return HS2_ERR_INVALID_ARG;
   if (!aligned16(Q_l) || !aligned16(K) || !aligned16(V) || !aligned16(O_part)) return HS2_ERR_INVALID_ARG;
   const SparseShard sh{pos0, ml_part};
   return run_sparse(p, Q_l, K, V, idx, count, idx_stride, 0, O_part, stream, &sh);

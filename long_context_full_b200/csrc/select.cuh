@@ -803,32 +803,42 @@ __global__ void __launch_bounds__(256) k_block_max(const float* scores, int64_t 
 }
 
 // Expands the selected blocks (ascending block ids) into their candidate
-// positions, then the window, the -1 padding and the count.
+// positions, then the window, the -1 padding and the count.  A row whose
+// geometry the block-max kernel rejected (more candidates than the score
+// stride, or more blocks than the block-max stride; already reported) gets
+// count 0 and all -1, so its output never depends on earlier scratch.
 __global__ void __launch_bounds__(256) k_block_expand(const int32_t* bsel, int nbsel_max,
                                                       const int64_t* qoff, const int64_t* kvoff, int B,
-                                                      int Hkv, int block, int window, int32_t* idx,
-                                                      int64_t idx_stride, int32_t* count) {
+                                                      int Hkv, int block, int window, int64_t stride,
+                                                      int64_t bstride, int32_t* idx, int64_t idx_stride,
+                                                      int32_t* count, int* err) {
   grid_dep_wait();  // the previous kernel on the stream has finished
   const int64_t r = blockIdx.x;
   const QueryRow q = query_row(qoff, kvoff, B, r / Hkv);
   int64_t nc = q.t - window + 1;
   if (nc < 0) nc = 0;
   const int64_t nb = (nc + block - 1) / block;
-  const int64_t nsel = nb < nbsel_max ? nb : nbsel_max;
+  const bool bad = nc > stride || nb > bstride;
+  int64_t nsel = bad ? 0 : (nb < nbsel_max ? nb : nbsel_max);
   int32_t* out = idx + r * idx_stride;
   const int32_t* bs = bsel + r * nbsel_max;
   int64_t ntok = 0;
   if (nsel > 0) {
     // every selected block but possibly the last (the highest id) is full
     const int64_t last = bs[nsel - 1];
-    const int64_t last_len = (last * block + block < nc ? block : nc - last * block);
-    ntok = (nsel - 1) * block + last_len;
-    for (int64_t i = threadIdx.x; i < ntok; i += blockDim.x) {
-      const int64_t bi = i / block, o = i % block;
-      out[i] = (int32_t)((int64_t)bs[bi] * block + o);
+    if (last < 0 || last >= nb) {  // not a block of this row: the selection did not run on it
+      if (threadIdx.x == 0) record_error(err, HS2_ERR_DEVICE_INPUT);
+      nsel = 0;
+    } else {
+      const int64_t last_len = (last * block + block < nc ? block : nc - last * block);
+      ntok = (nsel - 1) * block + last_len;
+      for (int64_t i = threadIdx.x; i < ntok; i += blockDim.x) {
+        const int64_t bi = i / block, o = i % block;
+        out[i] = (int32_t)((int64_t)bs[bi] * block + o);
+      }
     }
   }
-  const int64_t wlen = q.t + 1 < window ? (q.t + 1 > 0 ? q.t + 1 : 0) : window;
+  const int64_t wlen = bad ? 0 : (q.t + 1 < window ? (q.t + 1 > 0 ? q.t + 1 : 0) : window);
   const int64_t w0 = q.t - wlen + 1;
   for (int64_t i = threadIdx.x; i < idx_stride - ntok; i += blockDim.x)
     out[ntok + i] = i < wlen ? (int32_t)(w0 + i) : -1;

@@ -140,6 +140,41 @@ def check_index_sets(gidx, gcnt, oidx, ocnt, oscores, t, k, window, what):
     return len(diff)
 
 
+def check_block_sets(gidx, gcnt, oidx, ocnt, oscores, t, n_blocks, block, window, what):
+    """End-to-end rule of the block path (the token rule lifted to blocks): the
+    window part is identical; the global part is a union of whole candidate
+    blocks (their positions below t - window + 1), ascending; and every block in
+    the symmetric difference of the GPU's and the oracle's block sets has an
+    oracle block score within TIE_REL * b* of b*, the n_blocks-th highest
+    eligible block score.  Counts then agree unless a near-tie swapped the
+    partial block at the window's edge for a whole one."""
+    wlen = min(t + 1, window)
+    assert list(gidx[gcnt - wlen:gcnt]) == list(oidx[ocnt - wlen:ocnt]), f"{what}: window differs"
+    assert np.all(gidx[gcnt:] == -1), f"{what}: padding"
+    nc = max(0, t - window + 1)
+    glob = np.asarray(gidx[:gcnt - wlen], np.int64)
+    assert np.all(np.diff(glob) > 0) and (glob.size == 0 or (glob[0] >= 0 and glob[-1] < nc)), \
+        f"{what}: global part not ascending candidates"
+    gb = sorted(set((glob // block).tolist()))
+    whole = np.concatenate([np.arange(b * block, min((b + 1) * block, nc)) for b in gb]) \
+        if gb else np.zeros(0, np.int64)
+    assert np.array_equal(glob, whole), f"{what}: blocks not kept whole"
+    ob = sorted(set((np.asarray(oidx[:ocnt - wlen], np.int64) // block).tolist()))
+    assert len(gb) == len(ob), f"{what}: {len(gb)} blocks != {len(ob)}"
+    diff = set(gb) ^ set(ob)
+    if not diff:
+        assert gcnt == ocnt, f"{what}: count {gcnt} != {ocnt}"
+        return 0
+    s = np.asarray(oscores[:nc], np.float64)
+    nb = (nc + block - 1) // block
+    bscore = np.array([s[b * block:min((b + 1) * block, nc)].max() for b in range(nb)])
+    bstar = np.sort(bscore)[::-1][n_blocks - 1]
+    for b in diff:
+        assert abs(bscore[b] - bstar) <= TIE_REL * bstar, \
+            f"{what}: block {b} (score {bscore[b]:.9g}) differs away from the threshold {bstar:.9g}"
+    return len(diff)
+
+
 def gpu_select_on(scores_rows: np.ndarray, ts, k=1024, window=128, block_mode=False,
                   n_blocks=16, block=64, stride=None):
     """Runs the GPU selection on given float32 score rows (one query row per

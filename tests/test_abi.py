@@ -139,3 +139,35 @@ def test_context_parallel_calls_reject_bad_arguments_on_the_host(lib):
                                  None) == hs2.HS2_ERR_UNSUPPORTED
     assert lib.hs2_cp_topk_merge(P(), 0, 1024, 128, 0x1000, 0x2000, 0x3000, 0x4000,
                                  None) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_empty_step_returns_ok_without_pointers(lib):
+    """total_q = 0: every call checks the problem and its scalars, launches
+    nothing and returns HS2_OK with null tensor and workspace pointers (no
+    device is touched, so this runs without a GPU)."""
+    P = lambda **kw: ctypes.byref(_problem(**dict(dict(total_q=0, B=2, total_kv=150), **kw)))
+    assert lib.hs2_full_attn_scores(P(), None, None, None, None, None, 128, None, 0, None) == hs2.HS2_OK
+    assert lib.hs2_full_attn_scores(P(max_q_len=0), None, None, None, None, None, 128, None, 0,
+                                    None) == hs2.HS2_OK
+    assert lib.hs2_topk_select(P(), None, 128, 1024, 128, None, None, None, 0, None) == hs2.HS2_OK
+    assert lib.hs2_block_select(P(), None, 128, 16, 64, 128, None, None, None, 0, None) == hs2.HS2_OK
+    assert lib.hs2_block_select_noalloc(P(), None, 128, 16, 64, 128, None, None, None) == hs2.HS2_OK
+    assert lib.hs2_sparse_attn(P(), None, None, None, None, None, 1152, None, None, 0, None) == hs2.HS2_OK
+    assert lib.hs2_swa_attn(P(), None, None, None, 128, None, None) == hs2.HS2_OK
+    assert lib.hs2_kv_append(P(), None, None, None, None, None) == hs2.HS2_OK
+    assert lib.hs2_cp_attn_partial(P(), None, None, None, None, None, None, 0, None) == hs2.HS2_OK
+    assert lib.hs2_cp_scores(P(), None, None, 128, None, 0, None) == hs2.HS2_OK
+    assert lib.hs2_cp_topk_local(P(), None, 128, 1024, 128, None, None, None, None, None,
+                                 None) == hs2.HS2_OK
+    assert lib.hs2_cp_topk_merge(P(), 2, 1024, 128, None, None, None, None, None) == hs2.HS2_OK
+    assert lib.hs2_cp_sparse_partial(P(), None, None, None, None, None, 1152, None, None, None,
+                                     None) == hs2.HS2_OK
+    # the scalar arguments are still checked
+    assert lib.hs2_topk_select(P(), None, 128, 0, 128, None, None, None, 0, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_block_select(P(), None, 128, 16, 0, 128, None, None, None, 0,
+                                None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_sparse_attn(P(), None, None, None, None, None, 0, None, None, 0,
+                               None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_swa_attn(P(), None, None, None, 0, None, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_full_attn_scores(P(Hq=7), None, None, None, None, None, 128, None, 0,
+                                    None) == hs2.HS2_ERR_INVALID_ARG

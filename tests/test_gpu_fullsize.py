@@ -7,8 +7,8 @@ import pytest
 
 import oracle
 import synth
-from tests.gpu_util import (GpuRun, OracleRows, check_O, check_index_sets, check_scores,
-                            gpu_select_on, to_f64)
+from tests.gpu_util import (GpuRun, OracleRows, check_O, check_block_sets, check_index_sets,
+                            check_scores, gpu_select_on, to_f64)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -41,7 +41,8 @@ def check_rows(w, rows, select="token"):
                     report["recall_ora"].append(len(needles & set(oi[:oc].tolist())) / len(needles))
             else:
                 oi, oc = oracle.block_select(sref[g], t, w.n_blocks, w.block, w.window)
-                assert cnt == oc
+                report["flips"] += check_block_sets(idx, cnt, oi, oc, sref[g], t, w.n_blocks,
+                                                    w.block, w.window, f"blocks {r}/{g}")
             sets.append(idx[:cnt])
         for l in range(w.n_layers):
             ref = ora.sparse(r, l, sets)

@@ -7,8 +7,8 @@ import torch
 import oracle
 import synth
 from long_context_full_b200 import hs2
-from tests.gpu_util import (GpuRun, OracleRows, check_O, check_index_sets, check_scores,
-                            gpu_select_on, to_f64)
+from tests.gpu_util import (GpuRun, OracleRows, check_O, check_block_sets, check_index_sets,
+                            check_scores, gpu_select_on, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -43,7 +43,9 @@ def full_check(w, select="token", rows=None, layers=True):
                 summ["flips"] += check_index_sets(idx[R], int(cnt[R]), oi, oc, sref[g], t, w.topk,
                                                   w.window, f"indices row {r} g {g}")
             else:
-                assert int(cnt[R]) == oc
+                summ["flips"] += check_block_sets(idx[R], int(cnt[R]), oi, oc, sref[g], t,
+                                                  w.n_blocks, w.block, w.window,
+                                                  f"blocks row {r} g {g}")
         if layers:
             sets = [idx[r * w.Hkv + g, :cnt[r * w.Hkv + g]] for g in range(w.Hkv)]
             for l in range(w.n_layers):
@@ -299,3 +301,63 @@ def test_host_checks_launch_nothing():
     assert e.value.status == hs2.HS2_ERR_WORKSPACE
     torch.cuda.synchronize()
     assert torch.equal(before, run.step.idx)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("q_lens", [[1, 0, 1, 0, 1, 0], [0, 5, 0, 1, 40, 0]],
+                         ids=["decode", "chunk"])
+def test_sequences_without_queries(dtype, q_lens):
+    """A batch mixing sequences with no query token (Tq_b = 0) with decode and
+    chunk sequences: every kernel skips the empty ones by their offsets, and the
+    others match the oracle through the whole path (scores, token and block
+    selection, the no-allocation block selection, sparse layers)."""
+    kv = [3000, 1800, 1300, 2500, 1500, 700]
+    w = synth.make_workload("noq", 97, dtype, 16, 2, 128, kv, q_lens, 2)
+    summ, out = full_check(w)
+    assert summ["flips"] == 0
+    summ, out = full_check(w, select="block")
+    # the no-allocation block selection gives the same result on the same scores
+    run = GpuRun(w, select="block")
+    o = run.run()
+    idx2 = torch.full_like(o.idx, 7777)
+    cnt2 = torch.full_like(o.count, 7777)
+    hs2.hs2_block_select_noalloc(run.step.problem, o.scores, run.step.stride, w.n_blocks, w.block,
+                                 w.window, idx2, cnt2)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    assert torch.equal(idx2, o.idx) and torch.equal(cnt2, o.count)
+
+
+def test_step_without_query_rows():
+    """total_q = 0: every call returns HS2_OK and writes nothing - buffers
+    handed in anyway keep their canary bytes."""
+    B, Hq, Hkv, D = 3, 16, 2, 128
+    kv_lens = [500, 300, 1200]
+    qo = torch.zeros(B + 1, dtype=torch.int64, device="cuda")
+    ko = torch.tensor(np.concatenate([[0], np.cumsum(kv_lens)]), dtype=torch.int64, device="cuda")
+    tkv = int(sum(kv_lens))
+    for dt, code in ((torch.bfloat16, hs2.HS2_BF16), (torch.float32, hs2.HS2_F32)):
+        for max_q in (0, 1, 4):
+            p = hs2.make_problem(B, Hq, Hkv, D, code, qo, ko, 0, tkv, max_q, max(kv_lens), 0.088)
+            K = torch.randn(tkv, Hkv, D, device="cuda").to(dt)
+            V = torch.randn(tkv, Hkv, D, device="cuda").to(dt)
+            Kc, Vc = K.clone(), V.clone()
+            Q = torch.randn(4, Hq, D, device="cuda").to(dt)
+            O = torch.full((4, Hq, D), 7.0, device="cuda").to(dt)
+            S = torch.full((8, 1216), 5.0, device="cuda")
+            idx = torch.full((8, 1152), 7777, dtype=torch.int32, device="cuda")
+            cnt = torch.full((8,), 7777, dtype=torch.int32, device="cuda")
+            ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+            canaries = [t.clone() for t in (O, S, idx, cnt)]
+            hs2.hs2_full_attn_scores(p, Q, K, V, O, S, 1216, ws)
+            hs2.hs2_topk_select(p, S, 1216, 1024, 128, idx, cnt, ws)
+            hs2.hs2_block_select(p, S, 1216, 16, 64, 128, idx, cnt, ws)
+            hs2.hs2_block_select_noalloc(p, S, 1216, 16, 64, 128, idx, cnt)
+            hs2.hs2_sparse_attn(p, Q, K, V, idx, cnt, 1152, O, ws)
+            hs2.hs2_swa_attn(p, Q, K, V, 128, O)
+            hs2.hs2_kv_append(p, Q[:, :Hkv], Q[:, :Hkv], K, V)
+            torch.cuda.synchronize()
+            assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+            for a, b in zip((O, S, idx, cnt), canaries):
+                assert torch.equal(a, b)
+            assert torch.equal(K, Kc) and torch.equal(V, Vc)
