@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-subrecords", action="store_true",
+                    help="skip the needle 1M, chunk 262K and ragged 16 records of the default run")
     ap.add_argument("--batch", type=int, default=BATCH,
                     help="sequences per GPU (smaller only for profiling captures)")
     ap.add_argument("--context", type=int, default=CONTEXT,
@@ -311,6 +313,141 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
+def time_steps(step, Q, K, V, QL, n_steps: int, local: int, barrier=lambda: None):
+    """Times exactly ``n_steps`` hybrid-block steps on the current stream with
+    CUDA events around the whole region and around each phase (full attention,
+    selection, the sparse layers).  Returns (elapsed ms, per-step phase ms
+    [n_steps, 3], clock record)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(stream)
+    for i in range(n_steps):
+        e = ev[i]
+        e[0].record(stream)
+        step.full_attention(Q, K, V)
+        e[1].record(stream)
+        step.select_tokens()
+        e[2].record(stream)
+        for layer in range(step.n_layers):
+            step.sparse_layer(layer, QL[layer], K, V)
+        e[3].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ph = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+                   for e in ev])
+    return start.elapsed_time(end), ph, clk
+
+
+def load_workload(w, select: str = "token"):
+    """Device copies of a synthetic bf16 workload and a HybridBlockStep for it."""
+    import torch
+    from long_context_full_b200.block import HybridBlockStep
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    Q, K, V = dev(w.q), dev(w.k), dev(w.v)
+    QL = [dev(x) for x in w.q_layers]
+    step = HybridBlockStep(w.Hq, w.Hkv, w.D, torch.bfloat16, w.q_lens, w.kv_lens, w.n_layers,
+                           k=TOPK, window=WINDOW, select=select)
+    return step, Q, K, V, QL
+
+
+def warm(step, Q, K, V, QL, n: int):
+    """``n`` untimed steps (at least 3), then a check of the device error word."""
+    import torch
+    from long_context_full_b200 import hs2
+    for _ in range(max(3, n)):
+        step.run(Q, K, V, QL)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+
+
+def needle_recall(w, idx, count):
+    """Needle recall per KV group of the GPU's index sets (idx / count of the
+    decode row) beside that of the oracle's own selection on its own scores."""
+    import oracle
+    import synth
+    G = w.Hq // w.Hkv
+    n = int(w.kv_lens[0])
+    t = n - 1
+    needles = set(w.needle_pos[0].tolist())
+    gpu, ora = [], []
+    for g in range(w.Hkv):
+        ks = synth.stored_to_f64(w.k[:n, g:g + 1], w.dtype)
+        vs = synth.stored_to_f64(w.v[:n, g:g + 1], w.dtype)
+        q = synth.stored_to_f64(w.q[0, g * G:(g + 1) * G], w.dtype)
+        _, _, _, P = oracle.full_attention_row(q, ks, vs, t, w.scale)
+        s = oracle.selection_scores(P, 1)[0]
+        oi, oc = oracle.topk_select(s, t, w.topk, w.window)
+        ora.append(len(needles & set(oi[:oc].tolist())) / len(needles))
+        gpu.append(len(needles & set(idx[g, :int(count[g])].tolist())) / len(needles))
+    return gpu, ora
+
+
+def subrecord(w, args, local, hbm, select_compare: bool = False, recall: bool = False):
+    """One more of the pages' workload shapes, timed like the headline (same
+    steps and warm-up, its own clock record): ms per step, phase times and its
+    roofline figures."""
+    import torch
+    from long_context_full_b200 import hs2
+    step, Q, K, V, QL = load_workload(w)
+    warm(step, Q, K, V, QL, args.warmup)
+    el, ph, clk = time_steps(step, Q, K, V, QL, args.steps, local)
+    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+    ms = el / args.steps
+    t_full, t_sel, t_sp = (float(x) for x in ph.mean(axis=0))
+    ab = workload_accounting(w, w.n_layers)
+    rec = {"workload": w.name, "query_tokens": ab["queries"], "context": int(w.kv_lens.max()),
+           "ms_per_step": ms, "query_tok_s": ab["queries"] / (ms * 1e-3),
+           "phase_ms": {"full_attn_scores": t_full, "topk_select": t_sel,
+                        f"sparse_attn_x{w.n_layers}": t_sp},
+           "clocks": clk}
+    if int(w.q_lens.max()) > 1:
+        tf, tf_kind = tensor_peak()
+        achieved = ab["flops"] / (t_full * 1e-3) / 1e12
+        rec["full_attn_tflops"] = achieved
+        rec["full_attn_frac_of_tensor_peak"] = achieved / tf
+        rec["tensor_peak"] = {"value": tf, "unit": "TFLOP/s", "kind": tf_kind}
+        rec["score_write_gbs"] = (ab["full"] - ab["kv"]) / (t_full * 1e-3) / 1e9
+    else:
+        step_gbs = ab["step"] / (ms * 1e-3) / 1e9
+        rec["algorithmic_bytes_per_step"] = ab["step"]
+        rec["step_gbs"] = step_gbs
+        rec["step_frac_of_hbm"] = step_gbs / hbm
+        rec["step_frac_of_8TBps"] = step_gbs / 8000.0
+        rec["full_attn_gbs"] = ab["full"] / (t_full * 1e-3) / 1e9
+        rec["full_attn_frac_of_hbm"] = rec["full_attn_gbs"] / hbm
+        ss = ab["select"] + w.n_layers * ab["sparse_layer"]
+        rec["select_sparse_gbs"] = ss / ((t_sel + t_sp) * 1e-3) / 1e9
+    if recall:
+        gpu, ora = needle_recall(w, step.idx.cpu().numpy(), step.count.cpu().numpy())
+        rec["needle_recall"] = {"gpu": gpu, "oracle": ora,
+                                "note": "per KV group; parity means equal index sets, not recall 1"}
+    if select_compare:
+        del step
+        bstep, Q, K, V, QL = load_workload(w, select="block")
+        warm(bstep, Q, K, V, QL, args.warmup)
+        bel, bph, bclk = time_steps(bstep, Q, K, V, QL, args.steps, local)
+        assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+        rec["block_select_path"] = {
+            "ms_per_step": bel / args.steps,
+            "phase_ms": {"full_attn_scores": float(bph[:, 0].mean()),
+                         "block_select": float(bph[:, 1].mean()),
+                         f"sparse_attn_x{w.n_layers}": float(bph[:, 2].mean())},
+            "clocks": bclk}
+    torch.cuda.synchronize()
+    return rec
+
+
 def run_multiblock(args, local: int, n_blocks: int = 4):
     """A decode step through ``n_blocks`` Hybrid Blocks, each with its own
     8 x 131072-token cache (8 GiB of K/V in all), replayed as one CUDA graph:
@@ -661,7 +798,6 @@ def main():
     import torch.distributed as dist
     import synth
     from long_context_full_b200 import hs2
-    from long_context_full_b200.block import HybridBlockStep
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
@@ -705,14 +841,7 @@ def main():
                  "chunk_256k": synth.chunk_256k}[args.workload]()
             workload = w.name
     batch = int(w.q_lens.sum())  # query tokens per step
-
-    def dev(a):
-        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
-
-    Q, K, V = dev(w.q), dev(w.k), dev(w.v)
-    QL = [dev(x) for x in w.q_layers]
-    step = HybridBlockStep(w.Hq, w.Hkv, w.D, torch.bfloat16, w.q_lens, w.kv_lens, w.n_layers,
-                           k=TOPK, window=WINDOW)
+    step, Q, K, V, QL = load_workload(w)
     n_layers = w.n_layers
     stream = torch.cuda.current_stream()
 
@@ -720,42 +849,15 @@ def main():
         if world > 1:
             dist.barrier()
 
-    # ---- warm-up
-    for _ in range(max(3, args.warmup)):
-        step.run(Q, K, V, QL)
-    torch.cuda.synchronize()
-    assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
-
-    # ---- device-timed region: exactly K steps, events per phase
+    # ---- warm-up, then the device-timed region: exactly K steps, events per phase
+    warm(step, Q, K, V, QL, args.warmup)
     Kst = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(Kst)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
-    barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    start.record(stream)
-    for i in range(Kst):
-        e = ev[i]
-        e[0].record(stream)
-        step.full_attention(Q, K, V)
-        e[1].record(stream)
-        step.select_tokens()
-        e[2].record(stream)
-        for layer in range(n_layers):
-            step.sparse_layer(layer, QL[layer], K, V)
-        e[3].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    barrier()
-    elapsed_ms = start.elapsed_time(end)
-    ph = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
-                   for e in ev])
+    elapsed_ms, ph, clk = time_steps(step, Q, K, V, QL, Kst, local, barrier)
     assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
     elapsed_ms = max_over_ranks(elapsed_ms, world, "cuda")
     ms_step = elapsed_ms / Kst
     value = job_throughput(batch, world, Kst, elapsed_ms)
+    launches = step.launches_per_step()
 
     ab = workload_accounting(w, n_layers)
     t_full = float(ph[:, 0].mean())
@@ -808,6 +910,57 @@ def main():
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     e2e_value = job_throughput(batch, world, E, e2e_ms)
 
+    # ---- end to end with the cache resident (a decode server's case): per step
+    # the queries of every layer and each new token's K/V row come from pinned
+    # host memory, the rows are appended with hs2_kv_append (the same bytes at
+    # the same positions, so the cache does not change), the step runs, and
+    # its outputs are read back
+    e2e_res = None
+    if int(w.q_lens.max()) == 1:
+        last = w.kv_offsets[1:] - 1
+        hKn, hVn = pin(np.ascontiguousarray(w.k[last])), pin(np.ascontiguousarray(w.v[last]))
+        Kn, Vn = torch.empty_like(hKn, device="cuda"), torch.empty_like(hVn, device="cuda")
+        h2d_res = sum(t.numel() * t.element_size() for t in [hQ, hKn, hVn] + hQL)
+
+        def e2e_resident_step():
+            for d_, h_ in zip([Q, Kn, Vn] + QL, [hQ, hKn, hVn] + hQL):
+                d_.copy_(h_, non_blocking=True)
+            hs2.hs2_kv_append(step.problem, Kn, Vn, K, V)
+            step.run(Q, K, V, QL)
+            for h_, d_ in zip(hout, outs):
+                h_.copy_(d_, non_blocking=True)
+
+        e2e_resident_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(E):
+            e2e_resident_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert hs2.hs2_get_last_device_error() == hs2.HS2_OK
+        res_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+        e2e_res = {"value": job_throughput(batch, world, E, res_ms), "unit": UNIT,
+                   "h2d_bytes_per_step": h2d_res, "d2h_bytes_per_step": d2h, "steps": E,
+                   "note": "K/V cache resident; the new tokens' K/V rows appended each step"}
+
+    # ---- the other workloads of the metric's range, one GPU, default run only
+    subs = None
+    if (world == 1 and args.workload == "decode_b8_128k" and workload == WORKLOAD
+            and not args.no_subrecords):
+        del hK, hV
+        step = None
+        Q = K = V = None
+        QL = []
+        torch.cuda.empty_cache()
+        subs = {}
+        subs["needle_1m"] = subrecord(synth.needle_1m(), args, local, hbm, recall=True)
+        torch.cuda.empty_cache()
+        subs["chunk_262k"] = subrecord(synth.chunk_256k(), args, local, hbm)
+        torch.cuda.empty_cache()
+        subs["ragged_16"] = subrecord(synth.ragged_16(), args, local, hbm, select_compare=True)
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "decode_b8_128k":
         cpu = cpu_baseline(w)
@@ -831,9 +984,13 @@ def main():
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E},
-            "gpu_launches": Kst * step.launches_per_step(),
+            "gpu_launches": Kst * launches,
             "clocks": clk,
         }
+        if e2e_res is not None:
+            line["e2e_resident_cache"] = e2e_res
+        if subs is not None:
+            line["workloads"] = subs
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
