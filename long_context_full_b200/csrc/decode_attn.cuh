@@ -11,13 +11,20 @@
 //      of every KV head is cut into P balanced ranges, one per CTA, regardless
 //      of sequence boundaries (ragged batches stay balanced).  A CTA streams its
 //      K/V rows once, writes the scaled logits x_hj of its keys, and keeps an
-//      online-softmax partial (m, l, O) per warp and per sequence piece.
-//   2. k_decode_combine: merges the partials of each (sequence, head) into the
-//      output O and the final softmax statistics (m_h, l_h).
-//   3. k_finalize_scores: s_g[j] = sum_{h in g} exp(x_hj - m_h) / l_h.
+//      online-softmax partial (m, l, O) per warp and sequence piece; the bf16
+//      pass folds its warps' partials into one per piece before it ends.
+//   2. k_decode_combine: one CTA per (sequence, head) merges the partials of
+//      the CTAs that read the sequence into the output O and the final softmax
+//      statistics (m_h, l_h).
+//   3. k_finalize_scores: s_g[j] = sum_{h in g} exp(x_hj - m_h) / l_h, over the
+//      same CTA ranges as the pass, newest keys first (the logits the pass wrote
+//      last are the ones most likely still in L2), staged by bulk copies.
 // The per-head logits must be stored because the score needs each head's final
 // statistics, which are only known after the whole cache has been read; storing
 // them (32 B per key and KV head at G = 8) is far cheaper than reading K twice.
+// Logits are laid out group-major, [Hkv][total_kv][Gp] with Gp = G rounded up to
+// a multiple of 4, so a CTA's logits are one span and every key's row starts
+// on a 16-byte boundary.
 #pragma once
 
 #include "common.cuh"
@@ -38,12 +45,16 @@ struct DecodeArgs {
   int B, Hq, Hkv, G, P;   // P: CTAs per KV head
   int64_t total_q, total_kv;
   float scale;
-  float* logits;          // [total_kv, Hq]
+  float* logits;          // [Hkv, total_kv, Gp]
+  int Gp;                 // G rounded up to a multiple of 4
+  int nw;                 // warp partials per piece that hold data: 1 (bf16, folded) or kDecWarps
   float* pm;              // [(P+B), Hkv, kDecWarps, G]
   float* pl;
   float* po;              // [(P+B), Hkv, kDecWarps, G, D]
   int* err;
 };
+
+__host__ __device__ constexpr int logit_pitch(int G) { return (G + 3) & ~3; }
 
 // Walks the pieces (sequence b, key range [s, e)) of CTA p's key range; for
 // each piece whose sequence has a query row, calls f(b, s, e, q0).
@@ -71,16 +82,16 @@ __device__ __forceinline__ void for_each_piece(const DecodeArgs& a, int p, F f) 
 // register transpose (movmatrix), so no shared-memory round trip for P.
 // Warp 4 is the producer: one lane issues TMA loads into an NST-deep ring.
 // ----------------------------------------------------------------------------
+// The streaming pass of one CTA (p, g): ``ring`` is the NST-stage K/V ring in
+// dynamic shared memory, ``lg`` / ``kstride`` where key j's G logits of group
+// g go (lg + j * kstride + head).  Every thread of the CTA calls it; it returns
+// once this thread's part is done (the producer lane after its last fill has
+// landed).  Returns false if a bounded wait ran out.
 template <int NST>
-__global__ void __launch_bounds__(32 * (kDecWarps + 1))
-    k_decode_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const __grid_constant__ DecodeArgs a) {
-  grid_dep_wait();  // the previous kernel on the stream has finished
-  extern __shared__ uint8_t dsmem[];
-  __shared__ __align__(8) uint64_t full_bar[NST];
-  __shared__ __align__(8) uint64_t empty_bar[NST];
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-
+__device__ __forceinline__ bool decode_stream_bf16(const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                                   const DecodeArgs& a, uint8_t* ring,
+                                                   uint64_t* full_bar, uint64_t* empty_bar,
+                                                   float* lg, int64_t kstride) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.x, g = blockIdx.y;
 
@@ -95,7 +106,7 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
 
   if (warp == kDecWarps) {
     // ------------------------------------------------------------ producer
-    if (lane != 0) return;
+    if (lane != 0) return true;
     const uint64_t pol = policy_evict_first();
     int stage = 0;
     uint32_t phase = 0;
@@ -113,10 +124,10 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
         uint8_t* sk = ring + stage * kDecStageBytes;
         uint8_t* sv = sk + 2 * 8192;
         const int key = static_cast<int>(k0);
-        tma_load_3d_hint(sk, &tmK, &full_bar[stage], 0, g, key, pol);
-        tma_load_3d_hint(sk + 8192, &tmK, &full_bar[stage], 64, g, key, pol);
-        tma_load_3d_hint(sv, &tmV, &full_bar[stage], 0, g, key, pol);
-        tma_load_3d_hint(sv + 8192, &tmV, &full_bar[stage], 64, g, key, pol);
+        tma_load_3d_hint(sk, tmK, &full_bar[stage], 0, g, key, pol);
+        tma_load_3d_hint(sk + 8192, tmK, &full_bar[stage], 64, g, key, pol);
+        tma_load_3d_hint(sv, tmV, &full_bar[stage], 0, g, key, pol);
+        tma_load_3d_hint(sv + 8192, tmV, &full_bar[stage], 64, g, key, pol);
         issued |= 1u << stage;
         last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -125,8 +136,11 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
     // drain: every fill this thread issued has landed before the CTA can exit
     for (int s = 0; s < NST; ++s)
       if ((issued >> s) & 1u)
-        if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) record_error(a.err, HS2_ERR_TIMEOUT);
-    return;
+        if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) {
+          record_error(a.err, HS2_ERR_TIMEOUT);
+          ok = false;
+        }
+    return ok;
   }
 
   // -------------------------------------------------------------- consumers
@@ -157,7 +171,6 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
     const int h0 = 2 * qd, h1 = 2 * qd + 1;  // this thread's two heads
-    float* lg = a.logits + (int64_t)g * a.G;
 
     for (int64_t k0 = s; k0 < e; k0 += kDecTile) {
       if (ok && !mbar_wait(&full_bar[stage], phase)) {
@@ -188,16 +201,16 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
         // logits are read back by the score finalize right after this pass:
         // ask L2 to keep them (the K/V stream is loaded evict-first)
         if (h1 < a.G && (a.G & 1) == 0) {  // even G: the pair is 8-byte aligned
-          if (vlo) st_hint_f2(lg + klo * a.Hq + h0, x0, x1, keep);
-          if (vhi) st_hint_f2(lg + khi * a.Hq + h0, x2, x3, keep);
+          if (vlo) st_hint_f2(lg + klo * kstride + h0, x0, x1, keep);
+          if (vhi) st_hint_f2(lg + khi * kstride + h0, x2, x3, keep);
         } else {
           if (h0 < a.G) {
-            if (vlo) st_hint_f1(lg + klo * a.Hq + h0, x0, keep);
-            if (vhi) st_hint_f1(lg + khi * a.Hq + h0, x2, keep);
+            if (vlo) st_hint_f1(lg + klo * kstride + h0, x0, keep);
+            if (vhi) st_hint_f1(lg + khi * kstride + h0, x2, keep);
           }
           if (h1 < a.G) {
-            if (vlo) st_hint_f1(lg + klo * a.Hq + h1, x1, keep);
-            if (vhi) st_hint_f1(lg + khi * a.Hq + h1, x3, keep);
+            if (vlo) st_hint_f1(lg + klo * kstride + h1, x1, keep);
+            if (vhi) st_hint_f1(lg + khi * kstride + h1, x3, keep);
           }
         }
         // online softmax over the 16 keys of this warp, per head (column)
@@ -262,7 +275,63 @@ __global__ void __launch_bounds__(32 * (kDecWarps + 1))
         a.po[(base + h1) * kD + d + 8] = o[mt][3];
       }
     }
+    // fold the four warps' partials of this piece into warp 0's slot: thread d
+    // of the consumers takes dimension d of every head (4x fewer partials for
+    // the combine to read)
+    named_barrier_sync(1, 32 * kDecWarps);  // every consumer warp's partial is written
+    {
+      const int d = threadIdx.x;
+      const int64_t w0 = (slot * a.Hkv + g) * kDecWarps * a.G;
+      float acc[8], mm[8], ll[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        acc[h] = 0.f;
+        mm[h] = NEG;
+        ll[h] = 0.f;
+        if (h < a.G) {
+          float mw[kDecWarps];
+#pragma unroll
+          for (int w = 0; w < kDecWarps; ++w) {
+            mw[w] = a.pm[w0 + w * a.G + h];
+            mm[h] = fmaxf(mm[h], mw[w]);
+          }
+#pragma unroll
+          for (int w = 0; w < kDecWarps; ++w) {
+            const float f = exp_shift(mw[w], mm[h]);
+            acc[h] = fmaf(f, a.po[(w0 + w * a.G + h) * kD + d], acc[h]);
+            ll[h] = fmaf(f, a.pl[w0 + w * a.G + h], ll[h]);
+          }
+        }
+      }
+      named_barrier_sync(1, 32 * kDecWarps);  // every read of the four slots is done
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        if (h < a.G) {
+          a.po[(w0 + h) * kD + d] = acc[h];
+          if (d == 0) {
+            a.pm[w0 + h] = mm[h];
+            a.pl[w0 + h] = ll[h];
+          }
+        }
+      }
+    }
   });
+  return ok;
+}
+
+// Split-context pass as its own launch (the combine and the score finalize
+// follow as separate kernels).
+template <int NST>
+__global__ void __launch_bounds__(32 * (kDecWarps + 1))
+    k_decode_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ DecodeArgs a) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full_bar[NST];
+  __shared__ __align__(8) uint64_t empty_bar[NST];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  decode_stream_bf16<NST>(&tmK, &tmV, a, ring, full_bar, empty_bar,
+                          a.logits + (int64_t)blockIdx.y * a.total_kv * a.Gp, a.Gp);
 }
 
 // ----------------------------------------------------------------------------
@@ -301,7 +370,7 @@ __global__ void __launch_bounds__(32 * kDecWarps) k_decode_f32(const __grid_cons
         dot = fmaf(q[h].z, kv.z, dot);
         dot = fmaf(q[h].w, kv.w, dot);
         const float x = warp_sum(dot) * a.scale;
-        if (lane == 0) a.logits[j * a.Hq + (int64_t)g * a.G + h] = x;
+        if (lane == 0) a.logits[((int64_t)g * a.total_kv + j) * a.Gp + h] = x;
         const float mn = fmaxf(m[h], x);
         const float al = exp_shift(m[h], mn);
         const float pr = expf(x - mn);
@@ -325,19 +394,28 @@ __global__ void __launch_bounds__(32 * kDecWarps) k_decode_f32(const __grid_cons
 }
 
 // ----------------------------------------------------------------------------
-// Combine: O and (m_h, 1/l_h) of each (sequence, head) from the per-warp partials
-// of every CTA whose key range meets the sequence.  Grid (B, Hkv, G), D
-// threads: thread i owns partial i for the max and the weights, then thread d
-// sums dimension d over all partials (independent, coalesced loads).
+// Combine: O and (m_h, 1/l_h) of one (sequence, head) per CTA from the partials
+// of every CTA whose key range meets the sequence (nw per CTA piece).  Eight
+// warps: the partials' maxima and weights are computed lane-parallel and kept
+// in shared memory, then warp w sums partials w, w + 8, ... with each lane on
+// four dimensions (16-byte loads, several partials in flight per lane).
 // ----------------------------------------------------------------------------
-constexpr int kCombStage = 64;  // partial rows staged in shared memory per round
+constexpr int kCombThreads = 256;
+constexpr int kCombCap = 1024;  // partial weights staged per round
 
 template <typename OT>
-__global__ void __launch_bounds__(kD) k_decode_combine(const __grid_constant__ DecodeArgs a, OT* O,
-                                                       float* ml) {
+__global__ void __launch_bounds__(kCombThreads) k_decode_combine(const __grid_constant__ DecodeArgs a, OT* O,
+                                                                 float* ml) {
   grid_dep_wait();  // the previous kernel on the stream has finished
-  const int b = blockIdx.x, g = blockIdx.y, hl = blockIdx.z, d = threadIdx.x;
-  if (b == 0 && g == 0 && hl == 0 && d == 0) {
+  __shared__ float wsh[kCombCap];
+  __shared__ float red[kCombThreads / 32];
+  __shared__ __align__(16) float4 osh[kCombThreads / 32][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NW = kCombThreads / 32;
+  const int64_t item = blockIdx.x;
+  const int b = (int)(item / a.Hq), h = (int)(item % a.Hq);
+  const int g = h / a.G, hl = h % a.G;
+  if (item == 0 && threadIdx.x == 0) {
     if (__ldg(a.kvoff + a.B) != a.total_kv || __ldg(a.qoff + a.B) != a.total_q)
       record_error(a.err, HS2_ERR_DEVICE_INPUT);
   }
@@ -345,7 +423,7 @@ __global__ void __launch_bounds__(kD) k_decode_combine(const __grid_constant__ D
   const int64_t qn = __ldg(a.qoff + b + 1) - q0;
   if (qn < 1) return;
   if (qn > 1 || q0 < 0 || q0 >= a.total_q) {
-    if (d == 0 && hl == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+    if (threadIdx.x == 0 && hl == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
     return;
   }
   const int64_t W = a.total_kv;
@@ -353,177 +431,253 @@ __global__ void __launch_bounds__(kD) k_decode_combine(const __grid_constant__ D
   int pf = 0, np = 0;
   if (ke > kb) {
     pf = split_owner(W, a.P, kb);
-    np = (split_owner(W, a.P, ke - 1) - pf + 1) * kDecWarps;
+    np = (split_owner(W, a.P, ke - 1) - pf + 1) * a.nw;
   }
-  __shared__ __align__(16) float so[kCombStage][kD];
-  __shared__ float sw[kCombStage], swl[kCombStage];
-  __shared__ float red[kD / 32];
-  // partial i = (CTA pf + i / warps, warp i % warps); CTAs with an empty range wrote nothing
-  auto pidx = [&](int i, bool* valid) -> int64_t {
-    const int p = pf + i / kDecWarps;
-    *valid = split_lo(W, a.P, p) < split_lo(W, a.P, p + 1);
-    return (((int64_t)(p + b) * a.Hkv + g) * kDecWarps + (i % kDecWarps)) * a.G + hl;
+  // partial i = (CTA pf + i / nw, warp i % nw)
+  auto pidx = [&](int i) -> int64_t {
+    return (((int64_t)(pf + i / a.nw + b) * a.Hkv + g) * kDecWarps + (i % a.nw)) * a.G + hl;
   };
+  auto valid = [&](int i) {  // CTAs with an empty range wrote nothing
+    const int p = pf + i / a.nw;
+    return split_lo(W, a.P, p) < split_lo(W, a.P, p + 1);
+  };
+  // ---- the maximum over the partials
   float M = -INFINITY;
-  for (int i = d; i < np; i += kD) {
-    bool v;
-    const int64_t pi = pidx(i, &v);
-    if (v) M = fmaxf(M, a.pm[pi]);
-  }
+  for (int i = threadIdx.x; i < np; i += kCombThreads)
+    if (valid(i)) M = fmaxf(M, __ldcg(a.pm + pidx(i)));
   M = warp_max(M);
-  if ((d & 31) == 0) red[d >> 5] = M;
+  if (lane == 0) red[warp] = M;
   __syncthreads();
-  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  float L = 0.f, acc = 0.f;
-  for (int c0 = 0; c0 < np; c0 += kCombStage) {
-    const int n = min(kCombStage, np - c0);
-    if (d < n) {
-      bool v;
-      const int64_t pi = pidx(c0 + d, &v);
-      const float w = v ? exp_shift(a.pm[pi], M) : 0.f;
-      sw[d] = w;
-      swl[d] = w != 0.f ? w * a.pl[pi] : 0.f;
-    }
-    // the n partial O rows, all copies in flight at once (zero rows skipped)
-    for (int e = d; e < n * (kD / 4); e += kD) {
-      const int i = e / (kD / 4), c = e % (kD / 4);
-      bool v;
-      const int64_t pi = pidx(c0 + i, &v);
-      cp_async16(&so[i][c * 4], a.po + pi * kD + c * 4, v ? 16 : 0);
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    for (int i = 0; i < n; ++i) {
-      acc = fmaf(so[i][d], sw[i], acc);
-      L += swl[i];
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
+  // ---- per round of kCombCap partials: weights, then the weighted O rows
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c0 = 0; c0 < np; c0 += kCombCap) {
+    const int n = min(kCombCap, np - c0);
+    for (int i = threadIdx.x; i < n; i += kCombThreads) {
+      float w = 0.f;
+      if (valid(c0 + i)) {
+        const int64_t pi = pidx(c0 + i);
+        w = exp_shift(__ldcg(a.pm + pi), M);
+        L = fmaf(w, __ldcg(a.pl + pi), L);
+      }
+      wsh[i] = w;
     }
     __syncthreads();
+    constexpr int U = 4;
+    for (int i0 = warp; i0 < n; i0 += NW * U) {
+      float4 o[U];
+      float wt[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * NW;
+        wt[u] = i < n ? wsh[i] : 0.f;
+        o[u] = wt[u] != 0.f ? __ldcg(reinterpret_cast<const float4*>(a.po + pidx(c0 + i) * kD) + lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        acc.x = fmaf(wt[u], o[u].x, acc.x);
+        acc.y = fmaf(wt[u], o[u].y, acc.y);
+        acc.z = fmaf(wt[u], o[u].z, acc.z);
+        acc.w = fmaf(wt[u], o[u].w, acc.w);
+      }
+    }
+    __syncthreads();  // wsh is refilled by the next round
   }
-  const int64_t row = q0 * a.Hq + (int64_t)g * a.G + hl;
-  O[row * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
-  if (d == 0) {  // (m_h, 1 / l_h): the score finalize multiplies
-    ml[row * 2] = M;
-    ml[row * 2 + 1] = L > 0.f ? 1.f / L : 0.f;
+  L = warp_sum(L);
+  osh[warp][lane] = acc;
+  __syncthreads();  // red[] is free again: the maxima were read before the rounds
+  if (lane == 0) red[warp] = L;
+  __syncthreads();
+  if (warp == 0) {
+    float Lt = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      Lt += red[w];
+      const float4 v = osh[w][lane];
+      o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+    }
+    const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+    const int64_t row = q0 * a.Hq + h;
+    OT* dst = O + row * kD + lane * 4;
+    dst[0] = from_f<OT>(o.x * inv);
+    dst[1] = from_f<OT>(o.y * inv);
+    dst[2] = from_f<OT>(o.z * inv);
+    dst[3] = from_f<OT>(o.w * inv);
+    if (lane == 0) {  // (m_h, 1 / l_h): the score finalize multiplies
+      ml[row * 2] = M;
+      ml[row * 2 + 1] = inv;
+    }
   }
 }
 
 // ----------------------------------------------------------------------------
 // Scores: s_g[j] = sum_{h in group g} exp(x_hj - m_h) / l_h, written to row
-// (query, g) at column j.  Persistent grid: block i handles key tiles i,
-// i + gridDim.x, ... of kFinKeys keys each (tile = (sequence, key block)).  A
-// tile's logits [keys x Hq] are one contiguous span; they are copied into
-// shared memory with 16-byte cp.async (row pitch Hq + 4 floats, so the per-key
-// reads below are free of bank conflicts), double-buffered so that the copy of
-// the next tile overlaps the exponentials of this one.  Thread j scores key j
-// of the tile for every KV head; the writes are coalesced along j.
+// (query, g) at column j.  Grid (P, Hkv): CTA (p, g) takes the key range of the
+// pass's CTA (p, g), its pieces last first and each piece's keys from the top
+// down, so the logits written last are read first.  Warp 4 (one lane) streams
+// the logits into a ring of kFinStages stages of kFinChunk keys with untiled
+// bulk copies (the TMA engine; the span of a chunk is contiguous, its start
+// 16-byte aligned since Gp is a multiple of 4); warps 0-3 score two keys per
+// thread per stage and write the scores, coalesced along j.
 // ----------------------------------------------------------------------------
-constexpr int kFinKeys = 128;
+constexpr int kFinChunk = 256;
+constexpr int kFinStages = 4;
+constexpr int kFinThreads = 32 * (kDecWarps + 1);
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Tile -> (sequence, first key); tiles cover ceil(max_len / kFinKeys) blocks
-// of every sequence, empty ones are skipped.
-__device__ __forceinline__ bool fin_tile(const DecodeArgs& a, int64_t tile, int ntile_seq, int* b,
-                                         int64_t* q0, int64_t* kb, int64_t* j0, int* nk) {
-  *b = (int)(tile / ntile_seq);
-  *j0 = (tile % ntile_seq) * kFinKeys;
-  *q0 = __ldg(a.qoff + *b);
-  if (__ldg(a.qoff + *b + 1) - *q0 < 1) return false;
-  *kb = __ldg(a.kvoff + *b);
-  const int64_t N = __ldg(a.kvoff + *b + 1) - *kb;
-  if (*j0 >= N) return false;
-  *nk = (int)(N - *j0 < kFinKeys ? N - *j0 : kFinKeys);
-  return true;
+__host__ __device__ constexpr size_t finalize_smem(int G) {
+  return (size_t)kFinStages * kFinChunk * logit_pitch(G) * sizeof(float);
 }
 
-__global__ void __launch_bounds__(kFinKeys) k_finalize_scores(const __grid_constant__ DecodeArgs a,
-                                                              const float* ml, float* scores,
-                                                              int64_t stride, int ntile_seq) {
-  grid_dep_wait();  // the previous kernel on the stream has finished
-  extern __shared__ __align__(16) float fsm[];  // 2 x [kFinKeys][Hq + 4] logits, [Hq][2] stats
-  const int Hq = a.Hq, pitch = Hq + 4;
-  const int64_t ntiles = (int64_t)a.B * ntile_seq;
-  float* buf[2] = {fsm, fsm + (size_t)kFinKeys * pitch};
-  float* fst = fsm + 2 * (size_t)kFinKeys * pitch;  // (m_h, 1 / l_h) of the tile's query
-  const bool vec = (Hq & 3) == 0;
-  const bool vec4 = vec && (a.G & 3) == 0;
-  const uint64_t dead = policy_evict_first();  // each logit is read once
+// Walks the pieces of CTA p's key range last first; f(b, s, e, q0) as for_each_piece.
+template <typename F>
+__device__ __forceinline__ void for_each_piece_rev(const DecodeArgs& a, int p, F f) {
+  const int64_t W = a.total_kv;
+  const int64_t lo = split_lo(W, a.P, p), hi = split_lo(W, a.P, p + 1);
+  if (lo >= hi) return;
+  for (int b = last_le(a.kvoff, a.B, hi - 1); b >= 0; --b) {
+    const int64_t kb = __ldg(a.kvoff + b), ke = __ldg(a.kvoff + b + 1);
+    if (ke <= lo) break;
+    const int64_t s = kb > lo ? kb : lo, e = ke < hi ? ke : hi;
+    if (s >= e) continue;
+    const int64_t q0 = __ldg(a.qoff + b), qn = __ldg(a.qoff + b + 1) - q0;
+    if (qn < 1) continue;
+    if (q0 < 0 || q0 >= a.total_q) continue;  // inconsistent offsets: reported by the combine
+    f(b, s, e, q0);
+  }
+}
 
-  // issue the copy of one tile into buffer k (all threads); a tile whose
-  // offsets disagree with the totals copies nothing and is reported
-  auto load_tile = [&](int64_t tile, int k) -> bool {
-    int b, nk;
-    int64_t q0, kb, j0;
-    if (!fin_tile(a, tile, ntile_seq, &b, &q0, &kb, &j0, &nk)) return false;
-    const int64_t N = __ldg(a.kvoff + b + 1) - kb;
-    if (q0 < 0 || q0 >= a.total_q || kb < 0 || kb + N > a.total_kv || N > stride) {
-      if (threadIdx.x == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
-      return false;
+// One untiled bulk copy global -> this CTA's shared memory with an L2 policy,
+// completion counted on ``bar``; 16-byte aligned addresses, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                               uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_constant__ DecodeArgs a,
+                                                                 const float* ml, float* scores,
+                                                                 int64_t stride) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
+  extern __shared__ __align__(128) float fring[];
+  __shared__ __align__(8) uint64_t full_bar[kFinStages], empty_bar[kFinStages];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = blockIdx.x, g = blockIdx.y;
+  const int G = a.G, Gp = a.Gp;
+  const float* lg = a.logits + (int64_t)g * a.total_kv * Gp;
+  const int stage_floats = kFinChunk * Gp;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFinStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kDecWarps);
     }
-    const float* src = a.logits + (kb + j0) * Hq;
-    float* dst = buf[k];
-    if (vec) {
-      const int per_key = Hq / 4;
-      for (int i = threadIdx.x; i < nk * per_key; i += kFinKeys) {
-        const int key = i / per_key, c = i % per_key;
-        cp_async16_hint(dst + key * pitch + c * 4, src + (int64_t)key * Hq + c * 4, dead);
-      }
-    } else {
-      for (int i = threadIdx.x; i < nk * Hq; i += kFinKeys) dst[(i / Hq) * pitch + i % Hq] = __ldg(src + i);
-    }
-    return true;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // a piece whose offsets disagree with the score stride or the cache is skipped
+  // by both roles alike
+  auto piece_ok = [&](int b) {
+    const int64_t kb = __ldg(a.kvoff + b), N = __ldg(a.kvoff + b + 1) - kb;
+    return kb >= 0 && N <= stride && kb + N <= a.total_kv;
   };
 
-  int64_t tile = blockIdx.x;
-  int cur = 0;
-  bool have = tile < ntiles && load_tile(tile, 0);
-  cp_async_commit();
-  while (tile < ntiles) {
-    const int64_t next = tile + gridDim.x;
-    // next non-empty tile goes into the other buffer while this one is scored
-    int64_t nt = next;
-    bool nhave = false;
-    while (nt < ntiles && !(nhave = load_tile(nt, cur ^ 1))) nt += gridDim.x;
-    cp_async_commit();
-    if (have) {
-      int b, nk;
-      int64_t q0, kb, j0;
-      fin_tile(a, tile, ntile_seq, &b, &q0, &kb, &j0, &nk);  // checked by load_tile
-      {
-        // (m_h, 1/l_h) -> (m_h * log2 e, 1/l_h): exp(x - m) = 2^(x log2 e - m log2 e)
-        for (int i = threadIdx.x; i < 2 * Hq; i += kFinKeys) {
-          const float v = __ldg(ml + q0 * Hq * 2 + i);
-          fst[i] = (i & 1) ? v : v * 1.4426950408889634f;
+  if (warp == kDecWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    const uint64_t dead = policy_evict_first();  // each logit is read once
+    int stage = 0;
+    uint32_t phase = 0, issued = 0, last_phase = 0;
+    bool ok = true;
+    for_each_piece_rev(a, p, [&](int b, int64_t s, int64_t e, int64_t q0) {
+      if (!piece_ok(b)) return;
+      for (int64_t top = e; top > s && ok; top -= kFinChunk) {
+        const int64_t j0 = top - kFinChunk > s ? top - kFinChunk : s;
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1)) {
+          record_error(a.err, HS2_ERR_TIMEOUT);
+          ok = false;
+          break;
         }
-        cp_async_wait_prev();  // this tile's copy has landed (the next may be in flight)
-        __syncthreads();
-        const int kj = threadIdx.x;
-        if (kj < nk) {
-          const float* x = buf[cur] + kj * pitch;
-          for (int g = 0; g < a.Hkv; ++g) {
+        const uint32_t bytes = (uint32_t)((top - j0) * Gp * sizeof(float));
+        mbar_arrive_expect_tx(&full_bar[stage], bytes);
+        bulk_load_hint(fring + stage * stage_floats, lg + j0 * Gp, bytes, &full_bar[stage], dead);
+        issued |= 1u << stage;
+        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == kFinStages) { stage = 0; phase ^= 1; }
+      }
+    });
+    // drain: every copy issued here has landed before the CTA can exit
+    for (int s = 0; s < kFinStages; ++s)
+      if ((issued >> s) & 1u)
+        if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) record_error(a.err, HS2_ERR_TIMEOUT);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  int stage = 0;
+  uint32_t phase = 0;
+  bool ok = true;
+  for_each_piece_rev(a, p, [&](int b, int64_t s, int64_t e, int64_t q0) {
+    if (!piece_ok(b)) {
+      if (threadIdx.x == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+      return;
+    }
+    const int64_t kb = __ldg(a.kvoff + b);
+    float mh[16], il[16];  // (m_h log2 e, 1 / l_h) of the group's heads
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      mh[i] = 0.f;
+      il[i] = 0.f;
+      if (i < G) {
+        const int64_t row = q0 * a.Hq + (int64_t)g * G + i;
+        mh[i] = __ldg(ml + row * 2) * kLog2e;
+        il[i] = __ldg(ml + row * 2 + 1);
+      }
+    }
+    float* out = scores + (q0 * a.Hkv + g) * stride - kb;  // indexed by packed key j
+    for (int64_t top = e; top > s; top -= kFinChunk) {
+      const int64_t j0 = top - kFinChunk > s ? top - kFinChunk : s;
+      if (ok && !mbar_wait(&full_bar[stage], phase)) {
+        record_error(a.err, HS2_ERR_TIMEOUT);
+        ok = false;
+      }
+      if (ok) {
+        const float* x = fring + stage * stage_floats;
+#pragma unroll
+        for (int u = 0; u < kFinChunk / (32 * kDecWarps); ++u) {
+          const int i = (int)(top - j0) - 1 - (u * 32 * kDecWarps + (int)threadIdx.x);
+          if (i >= 0) {
+            const float* xr = x + i * Gp;
             float sc = 0.f;
-            if (vec4) {  // 16-byte reads: the row pitch of 9 x 16 bytes spreads 8 lanes over all banks
-              for (int h = g * a.G; h < (g + 1) * a.G; h += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(x + h);
-                sc = fmaf(ex2_approx(fmaf(v.x, kLog2e, -fst[2 * h])), fst[2 * h + 1], sc);
-                sc = fmaf(ex2_approx(fmaf(v.y, kLog2e, -fst[2 * h + 2])), fst[2 * h + 3], sc);
-                sc = fmaf(ex2_approx(fmaf(v.z, kLog2e, -fst[2 * h + 4])), fst[2 * h + 5], sc);
-                sc = fmaf(ex2_approx(fmaf(v.w, kLog2e, -fst[2 * h + 6])), fst[2 * h + 7], sc);
-              }
+            if (Gp == 8) {
+              const float4 v0 = reinterpret_cast<const float4*>(xr)[0];
+              const float4 v1 = reinterpret_cast<const float4*>(xr)[1];
+              const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+              for (int hh = 0; hh < 8; ++hh)
+                if (hh < G) sc = fmaf(ex2_approx(fmaf(v[hh], kLog2e, -mh[hh])), il[hh], sc);
             } else {
-              for (int h = g * a.G; h < (g + 1) * a.G; ++h)
-                sc = fmaf(ex2_approx(fmaf(x[h], kLog2e, -fst[2 * h])), fst[2 * h + 1], sc);
+#pragma unroll
+              for (int hh = 0; hh < 16; ++hh)
+                if (hh < G) sc = fmaf(ex2_approx(fmaf(xr[hh], kLog2e, -mh[hh])), il[hh], sc);
             }
-            scores[(q0 * a.Hkv + g) * stride + j0 + kj] = sc;
+            out[j0 + i] = sc;
           }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[stage]);
+      if (++stage == kFinStages) { stage = 0; phase ^= 1; }
     }
-    __syncthreads();  // buffer ``cur`` is free again
-    tile = nt;
-    have = nhave;
-    cur ^= 1;
-  }
-  cp_async_wait_all_groups();
+  });
 }
 
 }  // namespace hs2

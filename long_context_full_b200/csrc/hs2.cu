@@ -71,7 +71,6 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 
 constexpr size_t kCpMergeSmem = (size_t)kCpMergeCap * 8 + (size_t)kCpPickCap * 4;
-size_t finalize_smem(int Hq) { return (2 * (size_t)kFinKeys * (Hq + 4) + 2 * (size_t)Hq) * sizeof(float); }
 std::mutex g_dev_mu;
 
 template <int G>
@@ -125,7 +124,7 @@ hs2_status device_info(DeviceInfo** out) {
                                        cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
     cudaGetLastError();  // a refused non-portable size is not an error
     if (cudaFuncSetAttribute(k_finalize_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)finalize_smem(kMaxHq)) != cudaSuccess)
+                             (int)finalize_smem(16)) != cudaSuccess)
       return HS2_ERR_CUDA;
     if (cudaFuncSetAttribute(k_cp_topk_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kCpMergeSmem) != cudaSuccess)
@@ -196,7 +195,7 @@ DecodePlan plan_decode(const hs2_problem* p, const DeviceInfo& dev, void* ws) {
   pl.P = (int)std::min(target, by_size);
   Carve c(ws);
   const size_t slots = (size_t)(pl.P + p->B) * p->Hkv * kDecWarps * G;
-  pl.logits = c.take<float>((size_t)p->total_kv * p->Hq);
+  pl.logits = c.take<float>((size_t)p->Hkv * p->total_kv * logit_pitch(G));
   pl.pm = c.take<float>(slots);
   pl.pl = c.take<float>(slots);
   pl.po = c.take<float>(slots * kD);
@@ -263,16 +262,11 @@ void launch_decode_f32(dim3 grid, cudaStream_t st, const DecodeArgs& a) {
 
 // Decode scores from the logits the split-context pass kept and the final
 // (m, 1/l) of every (query, head).
-hs2_status launch_finalize(const hs2_problem* p, const DeviceInfo& dev, const DecodeArgs& a,
+hs2_status launch_finalize(const hs2_problem* p, const DeviceInfo&, const DecodeArgs& a,
                            const float* ml, float* scores, int64_t stride, cudaStream_t st) {
-  if (p->max_kv_len <= 0) return HS2_OK;
-  const int ntile_seq = (int)((p->max_kv_len + kFinKeys - 1) / kFinKeys);
-  const int64_t ntiles = (int64_t)p->B * ntile_seq;
-  int per_sm = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_finalize_scores, kFinKeys, finalize_smem(p->Hq));
-  const int64_t grid = std::min<int64_t>(ntiles, (int64_t)std::max(1, per_sm) * dev.sms);
-  launch(k_finalize_scores, dim3((unsigned)grid), dim3(kFinKeys), finalize_smem(p->Hq), st, 0, a, ml, scores, stride,
-         ntile_seq);
+  if (p->max_kv_len <= 0 || p->total_kv <= 0) return HS2_OK;
+  launch(k_finalize_scores, dim3((unsigned)a.P, (unsigned)p->Hkv), dim3(kFinThreads), finalize_smem(a.G), st, 0, a,
+         ml, scores, stride);
   return launch_status();
 }
 
@@ -290,16 +284,19 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
   a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = p->Hq / p->Hkv; a.P = pl.P;
   a.total_q = p->total_q; a.total_kv = p->total_kv; a.scale = p->scale;
   a.logits = pl.logits; a.pm = pl.pm; a.pl = pl.pl; a.po = pl.po; a.err = dev.err;
+  a.Gp = logit_pitch(a.G);
+  a.nw = p->dtype == HS2_BF16 ? 1 : kDecWarps;  // the bf16 pass folds its warps' partials
   const dim3 grid(pl.P, p->Hkv);
+  const dim3 cgrid((unsigned)((int64_t)p->B * p->Hq));
   if (p->dtype == HS2_BF16) {
     CUtensorMap mk, mv;
     if (encode_kv_map(&mk, K, p) != HS2_OK || encode_kv_map(&mv, V, p) != HS2_OK) return HS2_ERR_CUDA;
     launch(k_decode_bf16<kDecStages>, dim3(grid), dim3(32 * (kDecWarps + 1)), kDecStages * kDecStageBytes + 1024, st, 0, mk, mv, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     if (partial_ml)
-      launch(k_decode_combine<float>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<float*>(O), partial_ml);
+      launch(k_decode_combine<float>, cgrid, dim3(kCombThreads), 0, st, 0, a, static_cast<float*>(O), partial_ml);
     else
-      launch(k_decode_combine<bf16>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<bf16*>(O), pl.ml);
+      launch(k_decode_combine<bf16>, cgrid, dim3(kCombThreads), 0, st, 0, a, static_cast<bf16*>(O), pl.ml);
   } else {
     const int G = a.G;
     if (G <= 1) launch_decode_f32<1>(grid, st, a);
@@ -308,7 +305,7 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     else if (G <= 8) launch_decode_f32<8>(grid, st, a);
     else launch_decode_f32<16>(grid, st, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    launch(k_decode_combine<float>, dim3(dim3(p->B, p->Hkv, a.G)), dim3(kD), 0, st, 0, a, static_cast<float*>(O),
+    launch(k_decode_combine<float>, cgrid, dim3(kCombThreads), 0, st, 0, a, static_cast<float*>(O),
            partial_ml ? partial_ml : pl.ml);
   }
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
@@ -746,6 +743,8 @@ hs2_status hs2_cp_scores(const hs2_problem* p, const float* ml, float* scores, i
   a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = p->Hq / p->Hkv; a.P = pl.P;
   a.total_q = p->total_q; a.total_kv = p->total_kv; a.scale = p->scale;
   a.logits = pl.logits; a.err = dev->err;
+  a.Gp = logit_pitch(a.G);
+  a.nw = p->dtype == HS2_BF16 ? 1 : kDecWarps;
   return launch_finalize(p, *dev, a, ml, scores, score_stride, static_cast<cudaStream_t>(stream));
 }
 

@@ -39,7 +39,9 @@ namespace cg = cooperative_groups;
 constexpr int kSpWarps = 4;
 constexpr int kSpCluster = 8;
 constexpr int kSpRowBytes = 272;  // 256-byte bf16 row + 16 bytes: conflict-free ldmatrix
-constexpr int kSpPiece = 160;     // gathered rows staged per round (10 slices of 16)
+constexpr int kSpPiece = 144;     // gathered rows staged per round (9 slices of 16: a
+                                  // 1152-entry list over 8 CTAs in one round, and two
+                                  // CTAs fit on an SM)
 
 struct SparseArgs {
   const void* Q;        // [total_q, Hq, D], this layer's queries
