@@ -315,18 +315,26 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 def time_steps(step, Q, K, V, QL, n_steps: int, local: int, barrier=lambda: None):
     """Times exactly ``n_steps`` hybrid-block steps on the current stream with
-    CUDA events around the whole region and around each phase (full attention,
-    selection, the sparse layers).  Returns (elapsed ms, per-step phase ms
-    [n_steps, 3], clock record)."""
+    CUDA events around the whole region only (the kernels of consecutive calls
+    overlap their launches; an event between them would serialise that), then
+    ``n_steps`` more with events around each phase (full attention, selection,
+    the sparse layers) for the breakdown.  Returns (elapsed ms of the first
+    region, per-step phase ms [n_steps, 3], clock record of the first region)."""
     import torch
     stream = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
     clocks.start()
     start.record(stream)
+    for _ in range(n_steps):
+        step.run(Q, K, V, QL)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_steps)]
     for i in range(n_steps):
         e = ev[i]
         e[0].record(stream)
@@ -337,10 +345,7 @@ def time_steps(step, Q, K, V, QL, n_steps: int, local: int, barrier=lambda: None
         for layer in range(step.n_layers):
             step.sparse_layer(layer, QL[layer], K, V)
         e[3].record(stream)
-    end.record(stream)
     torch.cuda.synchronize()
-    clk = clocks.stop()
-    barrier()
     ph = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
                    for e in ev])
     return start.elapsed_time(end), ph, clk

@@ -6,19 +6,20 @@
 // builds the KV cache and decides which tokens are important) and "Xiaomi
 // Unveils HySparse2 for Faster Long-Context AI", section "Two-Level KV Sharing".
 //
-// Three launches:
+// Two launches:
 //   1. k_decode_bf16 / k_decode_f32: split-context pass.  The packed key space
 //      of every KV head is cut into P balanced ranges, one per CTA, regardless
 //      of sequence boundaries (ragged batches stay balanced).  A CTA streams its
 //      K/V rows once, writes the scaled logits x_hj of its keys, and keeps an
 //      online-softmax partial (m, l, O) per warp and sequence piece; the bf16
 //      pass folds its warps' partials into one per piece before it ends.
-//   2. k_decode_combine: one CTA per (sequence, head) merges the partials of
-//      the CTAs that read the sequence into the output O and the final softmax
-//      statistics (m_h, l_h).
-//   3. k_finalize_scores: s_g[j] = sum_{h in g} exp(x_hj - m_h) / l_h, over the
-//      same CTA ranges as the pass, newest keys first (the logits the pass wrote
-//      last are the ones most likely still in L2), staged by bulk copies.
+//   2. k_finalize_scores: merges the partials of every (sequence, head) into
+//      the output O, and computes s_g[j] = sum_{h in g} exp(x_hj - m_h) / l_h
+//      over the same CTA ranges as the pass, newest keys first (the logits the
+//      pass wrote last are the ones most likely still in L2), staged by bulk
+//      copies while the merge runs.
+// (k_decode_combine, the merge alone with float O and (m_h, 1/l_h) out, serves
+// the context-parallel partial pass.)
 // The per-head logits must be stored because the score needs each head's final
 // statistics, which are only known after the whole cache has been read; storing
 // them (32 B per key and KV head at G = 8) is far cheaper than reading K twice.
@@ -517,18 +518,25 @@ __global__ void __launch_bounds__(kCombThreads) k_decode_combine(const __grid_co
 }
 
 // ----------------------------------------------------------------------------
+// Finish of the decode call: the combine and the scores in one launch.
 // Scores: s_g[j] = sum_{h in group g} exp(x_hj - m_h) / l_h, written to row
 // (query, g) at column j.  Grid (P, Hkv): CTA (p, g) takes the key range of the
 // pass's CTA (p, g), its pieces last first and each piece's keys from the top
-// down, so the logits written last are read first.  Warp 4 (one lane) streams
+// down, so the logits written last are read first.  Warp 8 (one lane) streams
 // the logits into a ring of kFinStages stages of kFinChunk keys with untiled
-// bulk copies (the TMA engine; the span of a chunk is contiguous, its start
-// 16-byte aligned since Gp is a multiple of 4); warps 0-3 score two keys per
-// thread per stage and write the scores, coalesced along j.
+// bulk copies (the TMA engine; a chunk's span is contiguous and starts on a
+// 16-byte boundary since Gp is a multiple of 4), from the start of the kernel.
+// Meanwhile warps 0-7:
+//   1. (ml_in == null) merge the partials of the (sequence, head) items
+//      c, c + P*Hkv, ... into O, as k_decode_combine does;
+//   2. for each piece: the final (m_h, l_h) of the group's G heads, from the
+//      partials (lane-parallel, one warp per head) or from ml_in;
+//   3. score two keys per thread per stage, the writes coalesced along j.
 // ----------------------------------------------------------------------------
-constexpr int kFinChunk = 256;
+constexpr int kFinChunk = 512;
 constexpr int kFinStages = 4;
-constexpr int kFinThreads = 32 * (kDecWarps + 1);
+constexpr int kFinWarps = 8;
+constexpr int kFinThreads = 32 * (kFinWarps + 1);
 constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ constexpr size_t finalize_smem(int G) {
@@ -548,7 +556,7 @@ __device__ __forceinline__ void for_each_piece_rev(const DecodeArgs& a, int p, F
     if (s >= e) continue;
     const int64_t q0 = __ldg(a.qoff + b), qn = __ldg(a.qoff + b + 1) - q0;
     if (qn < 1) continue;
-    if (q0 < 0 || q0 >= a.total_q) continue;  // inconsistent offsets: reported by the combine
+    if (q0 < 0 || q0 >= a.total_q) continue;  // inconsistent offsets: reported with the O items
     f(b, s, e, q0);
   }
 }
@@ -564,21 +572,83 @@ __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint3
       : "memory");
 }
 
-__global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_constant__ DecodeArgs a,
-                                                                 const float* ml, float* scores,
+// The CTAs whose key range meets sequence b: [*pf, *pf + *pn).
+__device__ __forceinline__ void seq_owners(const DecodeArgs& a, int b, int* pf, int* pn) {
+  const int64_t W = a.total_kv;
+  const int64_t kb = __ldg(a.kvoff + b), ke = __ldg(a.kvoff + b + 1);
+  *pf = 0;
+  *pn = 0;
+  if (ke > kb) {
+    *pf = split_owner(W, a.P, kb);
+    *pn = split_owner(W, a.P, ke - 1) - *pf + 1;
+  }
+}
+
+// Index of partial i (= CTA pf + i / nw, warp i % nw) of (sequence b, KV head
+// g, head hl); -1 for a CTA with an empty range (it wrote nothing).
+__device__ __forceinline__ int64_t partial_at(const DecodeArgs& a, int b, int g, int hl, int pf, int i) {
+  const int p = pf + i / a.nw;
+  if (split_lo(a.total_kv, a.P, p) >= split_lo(a.total_kv, a.P, p + 1)) return -1;
+  return (((int64_t)(p + b) * a.Hkv + g) * kDecWarps + (i % a.nw)) * a.G + hl;
+}
+
+// Final (m, l) of one head from its np partials; one warp, every lane returns it.
+__device__ __forceinline__ void head_stats(const DecodeArgs& a, int b, int g, int hl, int pf, int np,
+                                           float* Mo, float* Lo) {
+  const int lane = threadIdx.x & 31;
+  constexpr int R = 4;  // partials a lane keeps in registers (np <= 128: one load each)
+  float mv[R], lv[R];
+  float M = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < R; ++u) {
+    const int i = u * 32 + lane;
+    mv[u] = -INFINITY;
+    lv[u] = 0.f;
+    const int64_t pi = i < np ? partial_at(a, b, g, hl, pf, i) : -1;
+    if (pi >= 0) {
+      mv[u] = __ldcg(a.pm + pi);
+      lv[u] = __ldcg(a.pl + pi);
+    }
+  }
+  for (int i = R * 32 + lane; i < np; i += 32) {
+    const int64_t pi = partial_at(a, b, g, hl, pf, i);
+    if (pi >= 0) M = fmaxf(M, __ldcg(a.pm + pi));
+  }
+#pragma unroll
+  for (int u = 0; u < R; ++u) M = fmaxf(M, mv[u]);
+  M = warp_max(M);
+  float L = 0.f;
+#pragma unroll
+  for (int u = 0; u < R; ++u) L = fmaf(exp_shift(mv[u], M), lv[u], L);
+  for (int i = R * 32 + lane; i < np; i += 32) {
+    const int64_t pi = partial_at(a, b, g, hl, pf, i);
+    if (pi >= 0) L = fmaf(exp_shift(__ldcg(a.pm + pi), M), __ldcg(a.pl + pi), L);
+  }
+  *Mo = M;
+  *Lo = warp_sum(L);
+}
+
+template <typename OT>
+__global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_constant__ DecodeArgs a, OT* O,
+                                                                 const float* ml_in, float* scores,
                                                                  int64_t stride) {
   grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ __align__(128) float fring[];
   __shared__ __align__(8) uint64_t full_bar[kFinStages], empty_bar[kFinStages];
+  __shared__ float wsh[kCombCap];
+  __shared__ __align__(16) float4 osh[kFinWarps][32];
+  __shared__ float red[kFinWarps];
+  __shared__ float cm[16], cl[16];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.x, g = blockIdx.y;
   const int G = a.G, Gp = a.Gp;
   const float* lg = a.logits + (int64_t)g * a.total_kv * Gp;
   const int stage_floats = kFinChunk * Gp;
+  constexpr int NC = 32 * kFinWarps;  // consumer threads
   if (threadIdx.x == 0) {
     for (int s = 0; s < kFinStages; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kDecWarps);
+      mbar_init(&empty_bar[s], kFinWarps);
     }
     fence_mbar_init();
   }
@@ -590,7 +660,7 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_co
     return kb >= 0 && N <= stride && kb + N <= a.total_kv;
   };
 
-  if (warp == kDecWarps) {
+  if (warp == kFinWarps) {
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
     const uint64_t dead = policy_evict_first();  // each logit is read once
@@ -621,7 +691,99 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_co
     return;
   }
 
-  // -------------------------------------------------------------- consumers
+  // ------------------------------------------------- consumers: 1. O items
+  if (!ml_in) {
+    const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x, nct = gridDim.x * gridDim.y;
+    if (cta == 0 && threadIdx.x == 0) {
+      if (__ldg(a.kvoff + a.B) != a.total_kv || __ldg(a.qoff + a.B) != a.total_q)
+        record_error(a.err, HS2_ERR_DEVICE_INPUT);
+    }
+    for (int64_t it = cta; it < (int64_t)a.B * a.Hq; it += nct) {
+      const int b = (int)(it / a.Hq), h = (int)(it % a.Hq);
+      const int gi = h / G, hl = h % G;
+      const int64_t q0 = __ldg(a.qoff + b), qn = __ldg(a.qoff + b + 1) - q0;
+      if (qn < 1) continue;  // a sequence without a query row (uniform over the CTA)
+      if (qn > 1 || q0 < 0 || q0 >= a.total_q) {
+        if (threadIdx.x == 0 && hl == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
+        continue;
+      }
+      int pf, pn;
+      seq_owners(a, b, &pf, &pn);
+      const int np = pn * a.nw;
+      float M = -INFINITY;
+      for (int i = threadIdx.x; i < np; i += NC) {
+        const int64_t pi = partial_at(a, b, gi, hl, pf, i);
+        if (pi >= 0) M = fmaxf(M, __ldcg(a.pm + pi));
+      }
+      M = warp_max(M);
+      if (lane == 0) red[warp] = M;
+      named_barrier_sync(1, NC);
+      M = red[0];
+#pragma unroll
+      for (int w = 1; w < kFinWarps; ++w) M = fmaxf(M, red[w]);
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c0 = 0; c0 < np; c0 += kCombCap) {
+        const int n = min(kCombCap, np - c0);
+        named_barrier_sync(1, NC);  // red[] / wsh[] of the step before are read
+        for (int i = threadIdx.x; i < n; i += NC) {
+          float w = 0.f;
+          const int64_t pi = partial_at(a, b, gi, hl, pf, c0 + i);
+          if (pi >= 0) {
+            w = exp_shift(__ldcg(a.pm + pi), M);
+            L = fmaf(w, __ldcg(a.pl + pi), L);
+          }
+          wsh[i] = w;
+        }
+        named_barrier_sync(1, NC);
+        constexpr int U = 4;
+        for (int i0 = warp; i0 < n; i0 += kFinWarps * U) {
+          float4 o[U];
+          float wt[U];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * kFinWarps;
+            wt[u] = i < n ? wsh[i] : 0.f;
+            const int pp = pf + (c0 + i) / a.nw;
+            const int64_t pi = (((int64_t)(pp + b) * a.Hkv + gi) * kDecWarps + ((c0 + i) % a.nw)) * G + hl;
+            o[u] = wt[u] != 0.f ? __ldcg(reinterpret_cast<const float4*>(a.po + pi * kD) + lane)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            acc.x = fmaf(wt[u], o[u].x, acc.x);
+            acc.y = fmaf(wt[u], o[u].y, acc.y);
+            acc.z = fmaf(wt[u], o[u].z, acc.z);
+            acc.w = fmaf(wt[u], o[u].w, acc.w);
+          }
+        }
+      }
+      L = warp_sum(L);
+      osh[warp][lane] = acc;
+      named_barrier_sync(1, NC);
+      if (lane == 0) red[warp] = L;
+      named_barrier_sync(1, NC);
+      if (warp == 0) {
+        float Lt = 0.f;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kFinWarps; ++w) {
+          Lt += red[w];
+          const float4 v = osh[w][lane];
+          o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+        }
+        const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+        OT* dst = O + (q0 * a.Hq + h) * kD + lane * 4;
+        dst[0] = from_f<OT>(o.x * inv);
+        dst[1] = from_f<OT>(o.y * inv);
+        dst[2] = from_f<OT>(o.z * inv);
+        dst[3] = from_f<OT>(o.w * inv);
+      }
+      named_barrier_sync(1, NC);  // osh / red are reused by the next item
+    }
+  }
+
+  // --------------------------------------- consumers: 2-3. statistics, scores
   int stage = 0;
   uint32_t phase = 0;
   bool ok = true;
@@ -631,17 +793,32 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_co
       return;
     }
     const int64_t kb = __ldg(a.kvoff + b);
+    if (ml_in) {
+      if (threadIdx.x < G) {
+        const int64_t row = q0 * a.Hq + (int64_t)g * G + threadIdx.x;
+        cm[threadIdx.x] = __ldg(ml_in + row * 2) * kLog2e;
+        cl[threadIdx.x] = __ldg(ml_in + row * 2 + 1);
+      }
+    } else {
+      int pf, pn;
+      seq_owners(a, b, &pf, &pn);
+      for (int hl = warp; hl < G; hl += kFinWarps) {
+        float M, L;
+        head_stats(a, b, g, hl, pf, pn * a.nw, &M, &L);
+        if (lane == 0) {
+          cm[hl] = M * kLog2e;
+          cl[hl] = L > 0.f ? 1.f / L : 0.f;
+        }
+      }
+    }
+    named_barrier_sync(1, NC);
     float mh[16], il[16];  // (m_h log2 e, 1 / l_h) of the group's heads
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      mh[i] = 0.f;
-      il[i] = 0.f;
-      if (i < G) {
-        const int64_t row = q0 * a.Hq + (int64_t)g * G + i;
-        mh[i] = __ldg(ml + row * 2) * kLog2e;
-        il[i] = __ldg(ml + row * 2 + 1);
-      }
+      mh[i] = i < G ? cm[i] : 0.f;
+      il[i] = i < G ? cl[i] : 0.f;
     }
+    named_barrier_sync(1, NC);  // cm / cl are rewritten by the next piece
     float* out = scores + (q0 * a.Hkv + g) * stride - kb;  // indexed by packed key j
     for (int64_t top = e; top > s; top -= kFinChunk) {
       const int64_t j0 = top - kFinChunk > s ? top - kFinChunk : s;
@@ -651,9 +828,10 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_co
       }
       if (ok) {
         const float* x = fring + stage * stage_floats;
+        const int n = (int)(top - j0);
 #pragma unroll
-        for (int u = 0; u < kFinChunk / (32 * kDecWarps); ++u) {
-          const int i = (int)(top - j0) - 1 - (u * 32 * kDecWarps + (int)threadIdx.x);
+        for (int u = 0; u < kFinChunk / NC; ++u) {
+          const int i = n - 1 - (u * NC + (int)threadIdx.x);
           if (i >= 0) {
             const float* xr = x + i * Gp;
             float sc = 0.f;

@@ -65,6 +65,7 @@ constexpr size_t kAlign = 256;
 struct DeviceInfo {
   bool ready = false;
   bool cluster16 = false;  // non-portable 16-CTA clusters allowed for the select kernel
+  bool sparse16 = false;   // ... and for the bf16 sparse kernel
   int sms = 0;
   int* err = nullptr;
 };
@@ -122,8 +123,12 @@ hs2_status device_info(DeviceInfo** out) {
                                        cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
                   cudaFuncSetAttribute(k_select_sampled<16>,
                                        cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    d.sparse16 = cudaFuncSetAttribute(k_sparse_bf16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                 cudaSuccess;
     cudaGetLastError();  // a refused non-portable size is not an error
-    if (cudaFuncSetAttribute(k_finalize_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(k_finalize_scores<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)finalize_smem(16)) != cudaSuccess ||
+        cudaFuncSetAttribute(k_finalize_scores<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)finalize_smem(16)) != cudaSuccess)
       return HS2_ERR_CUDA;
     if (cudaFuncSetAttribute(k_cp_topk_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -262,11 +267,15 @@ void launch_decode_f32(dim3 grid, cudaStream_t st, const DecodeArgs& a) {
 
 // Decode scores from the logits the split-context pass kept and the final
 // (m, 1/l) of every (query, head).
-hs2_status launch_finalize(const hs2_problem* p, const DeviceInfo&, const DecodeArgs& a,
-                           const float* ml, float* scores, int64_t stride, cudaStream_t st) {
+// The finish of a decode call: O (when ``O`` is given: merged from the
+// partials, as are the statistics) and the scores (statistics from ``ml_in``
+// when it is given).
+template <typename OT>
+hs2_status launch_finalize(const hs2_problem* p, const DecodeArgs& a, OT* O, const float* ml_in, float* scores,
+                           int64_t stride, cudaStream_t st) {
   if (p->max_kv_len <= 0 || p->total_kv <= 0) return HS2_OK;
-  launch(k_finalize_scores, dim3((unsigned)a.P, (unsigned)p->Hkv), dim3(kFinThreads), finalize_smem(a.G), st, 0, a,
-         ml, scores, stride);
+  launch(k_finalize_scores<OT>, dim3((unsigned)a.P, (unsigned)p->Hkv), dim3(kFinThreads), finalize_smem(a.G), st,
+         0, a, O, ml_in, scores, stride);
   return launch_status();
 }
 
@@ -293,10 +302,8 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     if (encode_kv_map(&mk, K, p) != HS2_OK || encode_kv_map(&mv, V, p) != HS2_OK) return HS2_ERR_CUDA;
     launch(k_decode_bf16<kDecStages>, dim3(grid), dim3(32 * (kDecWarps + 1)), kDecStages * kDecStageBytes + 1024, st, 0, mk, mv, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    if (partial_ml)
-      launch(k_decode_combine<float>, cgrid, dim3(kCombThreads), 0, st, 0, a, static_cast<float*>(O), partial_ml);
-    else
-      launch(k_decode_combine<bf16>, cgrid, dim3(kCombThreads), 0, st, 0, a, static_cast<bf16*>(O), pl.ml);
+    if (!partial_ml) return launch_finalize(p, a, static_cast<bf16*>(O), nullptr, scores, stride, st);
+    launch(k_decode_combine<float>, cgrid, dim3(kCombThreads), 0, st, 0, a, static_cast<float*>(O), partial_ml);
   } else {
     const int G = a.G;
     if (G <= 1) launch_decode_f32<1>(grid, st, a);
@@ -305,12 +312,10 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
     else if (G <= 8) launch_decode_f32<8>(grid, st, a);
     else launch_decode_f32<16>(grid, st, a);
     if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    launch(k_decode_combine<float>, cgrid, dim3(kCombThreads), 0, st, 0, a, static_cast<float*>(O),
-           partial_ml ? partial_ml : pl.ml);
+    if (!partial_ml) return launch_finalize(p, a, static_cast<float*>(O), nullptr, scores, stride, st);
+    launch(k_decode_combine<float>, cgrid, dim3(kCombThreads), 0, st, 0, a, static_cast<float*>(O), partial_ml);
   }
-  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  if (partial_ml) return HS2_OK;
-  return launch_finalize(p, dev, a, pl.ml, scores, stride, st);
+  return launch_status();
 }
 
 
@@ -594,6 +599,9 @@ hs2_status run_sparse(const hs2_problem* p, const void* Q_l, const void* K, cons
   if (p->dtype == HS2_BF16 && rows >= 4 * (int64_t)dev->sms && !shard) {
     // many rows (a chunk of queries): one CTA per row, no cluster
     e = launch(k_sparse_rows_bf16, dim3((unsigned)rows), dim3(32 * kSrWarps), kSrSmem, st, 0, a);
+  } else if (p->dtype == HS2_BF16 && dev->sparse16 && rows * 16 <= (int64_t)dev->sms) {
+    // few rows (a small decode batch): 16 CTAs per row, half the gathers each
+    e = launch_cluster(k_sparse_bf16, (unsigned)(rows * 16), 32 * kSpWarps, kSpSmem, 16, st, a);
   } else if (p->dtype == HS2_BF16) {
     e = launch_cluster(k_sparse_bf16, ctas, 32 * kSpWarps, kSpSmem, kSpCluster, st, a);
   } else {
@@ -745,7 +753,8 @@ hs2_status hs2_cp_scores(const hs2_problem* p, const float* ml, float* scores, i
   a.logits = pl.logits; a.err = dev->err;
   a.Gp = logit_pitch(a.G);
   a.nw = p->dtype == HS2_BF16 ? 1 : kDecWarps;
-  return launch_finalize(p, *dev, a, ml, scores, score_stride, static_cast<cudaStream_t>(stream));
+  return launch_finalize(p, a, static_cast<float*>(nullptr), ml, scores, score_stride,
+                         static_cast<cudaStream_t>(stream));
 }
 
 hs2_status hs2_cp_merge(int64_t rows, int32_t R, const float* O_parts, const float* ml_parts, int32_t dtype,

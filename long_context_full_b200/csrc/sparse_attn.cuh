@@ -37,7 +37,7 @@ namespace hs2 {
 namespace cg = cooperative_groups;
 
 constexpr int kSpWarps = 4;
-constexpr int kSpCluster = 8;
+constexpr int kSpCluster = 8;     // CTAs per row (16 when the rows are few)
 constexpr int kSpRowBytes = 272;  // 256-byte bf16 row + 16 bytes: conflict-free ldmatrix
 constexpr int kSpPiece = 144;     // gathered rows staged per round (9 slices of 16: a
                                   // 1152-entry list over 8 CTAs in one round, and two
@@ -115,12 +115,14 @@ __device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& 
 }
 
 // Partials received by the CTA that finishes a head: one slot per source CTA
-// and per owned head (heads h with h % cs == rank; at most kSpOwned of them).
-constexpr int kSpOwned = 2;
+// and per owned head (heads h with h % cs == rank), slot (c, s) at index
+// c * (kSpSlots / cs) + s.  A cluster of cs CTAs (8 or 16) leaves each CTA at
+// most kSpSlots / cs heads for G <= 16.
+constexpr int kSpSlots = 16;
 struct SpRecv {
-  float m[kSpCluster][kSpOwned];
-  float l[kSpCluster][kSpOwned];
-  float o[kSpCluster][kSpOwned][kD];
+  float m[kSpSlots];
+  float l[kSpSlots];
+  float o[kSpSlots][kD];
 };
 
 // One untiled bulk copy (the TMA engine, no tensor map) of ``bytes`` from
@@ -149,7 +151,7 @@ __device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_
                                                      const float* wo, SpRecv& recv) {
   __shared__ float wt[kSpWarps * GMAX];        // warp weights per head
   __shared__ float hm[GMAX], hl[GMAX];         // this CTA's (M, L) per head
-  __shared__ float ct[kSpOwned][kSpCluster];   // source-CTA weights per owned head
+  __shared__ float ct[kSpSlots];               // source-CTA weights per owned head
   const int d = threadIdx.x;
   if (d < a.G) {
     const int h = d;
@@ -170,21 +172,22 @@ __device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_
 #pragma unroll
     for (int w = 0; w < kSpWarps; ++w) acc = fmaf(wo[(w * GMAX + h) * kD + d], wt[w * GMAX + h], acc);
     SpRecv* dst = cl.map_shared_rank(&recv, h % cs);
-    const int slot = h / cs;
-    dst->o[rank][slot][d] = acc;
+    const int at = rank * (kSpSlots / cs) + h / cs;
+    dst->o[at][d] = acc;
     if (d == 0) {
-      dst->m[rank][slot] = hm[h];
-      dst->l[rank][slot] = hl[h];
+      dst->m[at] = hm[h];
+      dst->l[at] = hl[h];
     }
   }
   cl.sync();
   // owned heads h = rank, rank + cs, ...: slot (h - rank) / cs
   const int nown = a.G > rank ? (a.G - rank + cs - 1) / cs : 0;
+  const int per = kSpSlots / cs;
   if (d < nown * cs) {
     const int slot = d / cs, c = d % cs;
     float M = -INFINITY;
-    for (int c2 = 0; c2 < cs; ++c2) M = fmaxf(M, recv.m[c2][slot]);
-    ct[slot][c] = exp_shift(recv.m[c][slot], M);
+    for (int c2 = 0; c2 < cs; ++c2) M = fmaxf(M, recv.m[c2 * per + slot]);
+    ct[d] = exp_shift(recv.m[c * per + slot], M);
   }
   __syncthreads();
   OT* O = static_cast<OT*>(a.O);
@@ -192,15 +195,15 @@ __device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_
     const int slot = h / cs;
     float L = 0.f, acc = 0.f;
     for (int c = 0; c < cs; ++c) {
-      const float e = ct[slot][c];
-      L = fmaf(recv.l[c][slot], e, L);
-      acc = fmaf(recv.o[c][slot][d], e, acc);
+      const float e = ct[slot * cs + c];
+      L = fmaf(recv.l[c * per + slot], e, L);
+      acc = fmaf(recv.o[c * per + slot][d], e, acc);
     }
     const int64_t orow = qi * a.Hq + (int64_t)g * a.G + h;
     O[orow * kD + d] = from_f<OT>(L > 0.f ? acc / L : 0.f);
     if (a.ml_out && d == 0) {
       float M = -INFINITY;
-      for (int c = 0; c < cs; ++c) M = fmaxf(M, recv.m[c][slot]);
+      for (int c = 0; c < cs; ++c) M = fmaxf(M, recv.m[c * per + slot]);
       a.ml_out[orow * 2] = M;
       a.ml_out[orow * 2 + 1] = L > 0.f ? 1.f / L : 0.f;
     }
