@@ -59,7 +59,6 @@ constexpr int kMaxDevices = 64;
 constexpr int kDecStages = 3;     // bf16 decode ring depth (2 CTAs per SM)
 constexpr int kMaxHq = 192;      // query heads the score finalize can stage
 constexpr int kSelSmemKeys = 16384;  // select: per-CTA slice kept in shared memory (64 KB)
-constexpr size_t kSpSmem = 2 * (size_t)kSpPiece * kSpRowBytes + kSpPiece * 8;  // sparse: rows + positions
 constexpr size_t kAlign = 256;
 
 struct DeviceInfo {
@@ -94,7 +93,7 @@ hs2_status device_info(DeviceInfo** out) {
                              dec_smem) != cudaSuccess)
       return HS2_ERR_CUDA;
     if (cudaFuncSetAttribute(k_sparse_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSpSmem) != cudaSuccess ||
+                             (int)kSpGatherSmem) != cudaSuccess ||
         cudaFuncSetAttribute(k_sparse_rows_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSrSmem) != cudaSuccess)
       return HS2_ERR_CUDA;
@@ -595,15 +594,20 @@ hs2_status run_sparse(const hs2_problem* p, const void* Q_l, const void* K, cons
     a.pos0 = shard->pos0; a.ml_out = shard->ml_out; a.o_f32 = 1;
   }
   const unsigned ctas = (unsigned)(rows * kSpCluster);
+  // the cluster kernel gathers rows through a 2-D tensor map of (position, KV head) rows
+  const bool map_fits = p->total_kv * p->Hkv < (int64_t(1) << 31);
   cudaError_t e;
-  if (p->dtype == HS2_BF16 && rows >= 4 * (int64_t)dev->sms && !shard) {
+  if (p->dtype == HS2_BF16 && ((rows >= 4 * (int64_t)dev->sms && !shard) || !map_fits)) {
     // many rows (a chunk of queries): one CTA per row, no cluster
     e = launch(k_sparse_rows_bf16, dim3((unsigned)rows), dim3(32 * kSrWarps), kSrSmem, st, 0, a);
-  } else if (p->dtype == HS2_BF16 && dev->sparse16 && rows * 16 <= (int64_t)dev->sms) {
-    // few rows (a small decode batch): 16 CTAs per row, half the gathers each
-    e = launch_cluster(k_sparse_bf16, (unsigned)(rows * 16), 32 * kSpWarps, kSpSmem, 16, st, a);
   } else if (p->dtype == HS2_BF16) {
-    e = launch_cluster(k_sparse_bf16, ctas, 32 * kSpWarps, kSpSmem, kSpCluster, st, a);
+    CUtensorMap mk, mv;
+    const int64_t map_rows = p->total_kv * p->Hkv;
+    if (encode_map2(&mk, K, map_rows, kD, 1) != HS2_OK || encode_map2(&mv, V, map_rows, kD, 1) != HS2_OK)
+      return HS2_ERR_CUDA;
+    // few rows (a small decode batch): 16 CTAs per row, half the gathers each
+    const int cs = (dev->sparse16 && rows * 16 <= (int64_t)dev->sms) ? 16 : kSpCluster;
+    e = launch(k_sparse_bf16, dim3((unsigned)(rows * cs)), dim3(32 * kSpWarps), kSpGatherSmem, st, cs, mk, mv, a);
   } else {
     const int G = a.G;
     if (G <= 1) e = launch_cluster(k_sparse_f32<1>, ctas, 32 * kSpWarps, 0, kSpCluster, st, a);

@@ -7,12 +7,13 @@
 // and selection) and "Token-Level Selection and Unified Local Access" (local and
 // global tokens come from the one shared cache, in a single sparse computation).
 //
-// Few rows (decode): one thread-block cluster of kSpCluster CTAs per (query,
-// KV group) row.  CTA c takes the c-th share of the row's index list and
-// reads those K/V rows - bf16: one bulk copy (the TMA engine) per 256-byte row
-// into shared memory; fp32: each warp loads its rows straight into registers,
-// 16 bytes per lane - runs an online softmax per warp (tensor cores for
-// bf16), folds its warps into one partial,
+// Few rows (decode): one thread-block cluster of 8 CTAs (16 when the rows are
+// few) per (query, KV group) row.  CTA c takes the c-th share of the row's
+// index list and reads those K/V rows - bf16: TMA gather4 instructions, four
+// rows of a 2-D (position, KV head) x 128 tensor map each, in 64-column halves
+// with the 128-byte swizzle; fp32: each warp loads its rows straight into
+// registers, 16 bytes per lane - runs an online softmax per warp (tensor cores
+// for bf16), folds its warps into one partial,
 // and the cluster merges the partials through distributed shared memory, CTA c
 // finishing the heads h = c mod kSpCluster after a single cluster barrier.  No
 // workspace, no global round trip, no atomics.
@@ -38,7 +39,7 @@ namespace cg = cooperative_groups;
 
 constexpr int kSpWarps = 4;
 constexpr int kSpCluster = 8;     // CTAs per row (16 when the rows are few)
-constexpr int kSpRowBytes = 272;  // 256-byte bf16 row + 16 bytes: conflict-free ldmatrix
+constexpr int kSpRowBytes = 272;  // fp32 / row kernels: 256-byte row + 16 bytes, conflict-free ldmatrix
 constexpr int kSpPiece = 144;     // gathered rows staged per round (9 slices of 16: a
                                   // 1152-entry list over 8 CTAs in one round, and two
                                   // CTAs fit on an SM)
@@ -125,14 +126,18 @@ struct SpRecv {
   float o[kSpSlots][kD];
 };
 
-// One untiled bulk copy (the TMA engine, no tensor map) of ``bytes`` from
-// global memory into this CTA's shared memory, completion counted on ``bar``.
-// Both addresses 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_load_row(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+constexpr int kSpHalfBytes = kSpPiece * 128;  // bf16 cluster kernel: 64 columns of the staged rows
+constexpr size_t kSpGatherSmem = 4 * (size_t)kSpHalfBytes + (size_t)kSpPiece * 8 + 1024;  // + alignment
+
+// Four rows of a 2-D tensor map (box: 64 columns x 1 row, 128-byte swizzle)
+// gathered by one TMA instruction into 4 x 128 bytes at ``dst``, completion
+// counted on ``bar``: rows r0..r3, columns c0 .. c0 + 63 (c0 a multiple of 64).
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0,
+                                            int r1, int r2, int r3) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
 }
 
@@ -214,9 +219,11 @@ __device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_
 // bf16: tensor-core S^T = K Q^T and O^T += V^T P^T per 16-key slice, the same
 // fragment scheme as the decode pass (P^T by one movmatrix transpose).
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_constant__ SparseArgs a) {
+__global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_constant__ CUtensorMap tmK,
+                                                                const __grid_constant__ CUtensorMap tmV,
+                                                                const __grid_constant__ SparseArgs a) {
   grid_dep_wait();  // the previous kernel on the stream has finished
-  extern __shared__ __align__(128) uint8_t sp_smem[];
+  extern __shared__ uint8_t sp_dyn[];
   __shared__ float wm[kSpWarps * 8], wl[kSpWarps * 8];
   __shared__ float wo[kSpWarps * 8 * kD];
   __shared__ SpRecv recv;
@@ -224,17 +231,19 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
   cg::cluster_group cl = cg::this_cluster();
   const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
   if (threadIdx.x == 0) {
-    mbar_init(&gbar[0], blockDim.x);  // every thread arrives with the bytes it copies
-    mbar_init(&gbar[1], blockDim.x);
+    mbar_init(&gbar[0], 1);  // thread 0 arrives with the bytes of the group
+    mbar_init(&gbar[1], 1);
     fence_mbar_init();
   }
   const SpRow s = sparse_row(a, rank, cs);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // staged rows: K and V, each as two [kSpPiece][128 B] halves (columns 0-63,
+  // 64-127) in the 128-byte swizzle of the tensor maps, bases 1024-aligned
+  uint8_t* sp_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sp_dyn) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = sp_smem;
-  uint8_t* sV = sp_smem + (size_t)kSpPiece * kSpRowBytes;
-  int64_t* spos = reinterpret_cast<int64_t*>(sp_smem + 2 * (size_t)kSpPiece * kSpRowBytes);
-  const bf16* K = static_cast<const bf16*>(a.K);
-  const bf16* V = static_cast<const bf16*>(a.V);
+  uint8_t* sV = sp_smem + 2 * (size_t)kSpHalfBytes;
+  int64_t* spos = reinterpret_cast<int64_t*>(sp_smem + 4 * (size_t)kSpHalfBytes);
+  const int64_t map_rows = a.total_kv * a.Hkv;  // rows of the 2-D maps: (position, KV head)
 
   const int r = lane >> 2, qd = lane & 3;
   const int h0 = 2 * qd, h1 = 2 * qd + 1;
@@ -264,52 +273,46 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
     for (int row = threadIdx.x; row < ntile * 16; row += blockDim.x)
       spos[row] = row < pn ? sparse_pos(a, s, p0 + row, true) : -1;
     __syncthreads();
-    // gather: one bulk copy per 256-byte K row and per V row (the TMA engine
-    // moves them, no per-16-byte requests); rows past pn or with an invalid
-    // index are zero-filled by plain stores.  Two copy groups on their own
-    // barriers: the first half of the slices is scored while the second half
-    // is still in flight.  Every thread arrives once per group with the bytes
-    // of its own copies, and no copy is issued before all have arrived.
+    // gather: one TMA gather4 per 4 rows and per 64-column half of K and of V
+    // (rows past pn or with an invalid index load a row of the sequence that
+    // is then masked out).  Two copy groups on their own barriers: the first
+    // half of the slices is scored while the second half is still in flight.
+    // Thread 0 arrives on each group with its byte count before any copy.
     const int nA = (ntile + 1) / 2;
-    for (int grp = 0; grp < 2; ++grp) {
-      const int lo = grp == 0 ? 0 : nA * 16, hi = grp == 0 ? nA * 16 : ntile * 16;
-      uint32_t bytes = 0;
-      for (int row = lo + (int)threadIdx.x; row < hi; row += blockDim.x)
-        if (spos[row] >= 0) bytes += 2 * kD * sizeof(bf16);
-      mbar_arrive_expect_tx(&gbar[grp], bytes);
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(&gbar[0], (uint32_t)(nA * 16) * 4u * 128u);
+      mbar_arrive_expect_tx(&gbar[1], (uint32_t)((ntile - nA) * 16) * 4u * 128u);
     }
     __syncthreads();
-    for (int grp = 0; grp < 2; ++grp) {
-      const int lo = grp == 0 ? 0 : nA * 16, hi = grp == 0 ? nA * 16 : ntile * 16;
-      for (int row = lo + (int)threadIdx.x; row < hi; row += blockDim.x) {
-        const int64_t pos = spos[row];
-        uint8_t* dk = sK + (size_t)row * kSpRowBytes;
-        uint8_t* dv = sV + (size_t)row * kSpRowBytes;
-        if (pos >= 0) {
-          const int64_t off = ((s.kv_start + pos) * a.Hkv + s.g) * kD;
-          bulk_load_row(dk, K + off, kD * sizeof(bf16), &gbar[grp]);
-          bulk_load_row(dv, V + off, kD * sizeof(bf16), &gbar[grp]);
-        } else {
+    for (int q = threadIdx.x; q < ntile * 4; q += blockDim.x) {
+      const int row0 = q * 4;
+      uint64_t* bar = &gbar[row0 < nA * 16 ? 0 : 1];
+      int rr[4];
 #pragma unroll
-          for (int c = 0; c < kD * (int)sizeof(bf16) / 16; ++c) {
-            reinterpret_cast<uint4*>(dk)[c] = make_uint4(0u, 0u, 0u, 0u);
-            reinterpret_cast<uint4*>(dv)[c] = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
+      for (int u = 0; u < 4; ++u) {
+        const int64_t pos = spos[row0 + u];
+        int64_t mr = (s.kv_start + (pos >= 0 ? pos : 0)) * a.Hkv + s.g;
+        mr = mr < 0 ? 0 : (mr >= map_rows ? map_rows - 1 : mr);
+        rr[u] = (int)mr;
       }
+      const uint32_t off = (uint32_t)row0 * 128u;
+      tma_gather4(sK + off, &tmK, bar, 0, rr[0], rr[1], rr[2], rr[3]);
+      tma_gather4(sK + kSpHalfBytes + off, &tmK, bar, 64, rr[0], rr[1], rr[2], rr[3]);
+      tma_gather4(sV + off, &tmV, bar, 0, rr[0], rr[1], rr[2], rr[3]);
+      tma_gather4(sV + kSpHalfBytes + off, &tmV, bar, 64, rr[0], rr[1], rr[2], rr[3]);
     }
     for (int half = 0; half < 2; ++half) {
       if (!mbar_wait(&gbar[half], (uint32_t)(piece & 1))) record_error(a.err, HS2_ERR_TIMEOUT);
-      __syncthreads();  // and the zero-filled rows of other threads are visible
       for (int st = (half == 0 ? 0 : nA) + warp; st < (half == 0 ? nA : ntile); st += kSpWarps) {
         float c[4] = {0.f, 0.f, 0.f, 0.f};
         {
           const int row = st * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const int chunk = kk * 2 + (lane >> 4);
+            const int chunk = (kk & 3) * 2 + (lane >> 4);
+            const uint32_t addr = skb + (kk >> 2) * kSpHalfBytes + row * 128 + ((chunk ^ (row & 7)) << 4);
             uint32_t a0, a1, a2, a3;
-            ldsm_x4(a0, a1, a2, a3, skb + row * kSpRowBytes + chunk * 16);
+            ldsm_x4(a0, a1, a2, a3, addr);
             mma_bf16(c, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
           }
         }
@@ -341,15 +344,16 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
         const int row = st * 16 + ((lane >> 4) & 1) * 8 + (lane & 7);
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          const int chunk = mt * 2 + ((lane >> 3) & 1);
+          const int chunk = (mt & 3) * 2 + ((lane >> 3) & 1);
+          const uint32_t addr = svb + (mt >> 2) * kSpHalfBytes + row * 128 + ((chunk ^ (row & 7)) << 4);
           uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(a0, a1, a2, a3, svb + row * kSpRowBytes + chunk * 16);
+          ldsm_x4_t(a0, a1, a2, a3, addr);
           mma_bf16(o[mt], a0, a1, a2, a3, b0, b1);
         }
       }
     }
     __syncthreads();  // the next piece overwrites the staged rows
-    fence_proxy_async_smem();  // ... by bulk copies after these reads and stores
+    fence_proxy_async_smem();  // ... by TMA copies after these reads
   }
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
