@@ -484,7 +484,9 @@ __device__ __forceinline__ void sel_block_find(const uint32_t* hist, int nb, int
 // the exact selection over the slices in global memory.  Either way the result
 // equals a full stable sort by (score desc, position asc).
 template <int CS>
-__global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_constant__ SelectArgs a,
+// CS = 16 runs only for few long rows (one CTA per SM): it may use twice the
+// registers, for twice the loads in flight in the collect pass.
+__global__ void __launch_bounds__(kSelThreads, CS == 16 ? 1 : 2) k_select_sampled(const __grid_constant__ SelectArgs a,
                                                                 int32_t* count) {
   grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ uint4 ss_dyn[];
@@ -560,43 +562,25 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_
   }
   if (threadIdx.x == 0) st.ns = 4 * ngroups;
   csync();
-  // the cluster's sample histogram (CS > 1: summed by every CTA into st.tot's
-  // space is too small, so into the selected-position buffer, reused later)
-  uint32_t* hs = st.h;
-  int total = CS == 1 ? st.ns : 0;
-  if (CS > 1) {
-    hs = reinterpret_cast<uint32_t*>(sel);
-#pragma unroll
-    for (int c = 0; c < CS; ++c) total += *cl.map_shared_rank(&st.ns, c);
-#pragma unroll
-    for (int q = 0; q < kSelBins / kSelThreads; q += 2) {
-      uint32_t v[2][CS];
-#pragma unroll
-      for (int e = 0; e < 2; ++e)
-#pragma unroll
-        for (int c = 0; c < CS; ++c)
-          v[e][c] = *cl.map_shared_rank(&st.h[threadIdx.x + (q + e) * kSelThreads], c);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        uint32_t sum = 0;
-#pragma unroll
-        for (int c = 0; c < CS; ++c) sum += v[e][c];
-        hs[threadIdx.x + (q + e) * kSelThreads] = sum;
-      }
-    }
-    __syncthreads();
-  }
+  // tau = the lower edge of the bin holding the rs-th largest sample of the
+  // row.  CS > 1: the cluster's sample histograms are reduce-scattered (CTA c
+  // sums bins [c*own, (c+1)*own) over the cluster) and every CTA finds the
+  // same bin from the totals; a row with fewer than rs samples keeps tau = 0.
   const float kr_f = (float)a.k / (float)rho;
   const int rs = (int)ceilf(kr_f + 4.f * sqrtf(kr_f)) + 8;
   uint32_t tau = 0u;
-  if (total >= rs) {
-    sel_block_find(hs, kSelBins, rs, st.wgt, &st.digit, &st.krem);
+  if constexpr (CS > 1) {
+    const int own = sel_reduce_bins<CS>(cl, st, kSelBins);
+    sel_find_digit<CS>(cl, st, own, rs);
+    tau = st.digit << 21;
+  } else if (st.ns >= rs) {
+    sel_block_find(st.h, kSelBins, rs, st.wgt, &st.digit, &st.krem);
     tau = st.digit << 21;
   }
 
   // ---- 2. collect every key >= tau of the slice (unordered)
   {
-    constexpr int kBatch = 8;
+    constexpr int kBatch = CS == 16 ? 16 : 8;
     const int64_t len4 = vec ? (len & ~int64_t(3)) : 0;
     auto keep = [&](uint32_t u, int64_t o) {
       if (u >= tau) {
