@@ -880,7 +880,7 @@ def main():
     else:
         achieved = ab["full"] / (t_full * 1e-3) / 1e9
         traffic = profiled_traffic(kernel_sources_hash()) if workload == WORKLOAD else None
-        roof = {"kernel": "hs2_full_attn_scores (decode pass + combine + score finalize)",
+        roof = {"kernel": "hs2_full_attn_scores (decode pass + O merge and score finalize: 2 kernels)",
                 "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "peak_kind": hbm_kind,
                 "traffic": traffic, "algorithmic_bytes": ab["full"],
