@@ -484,9 +484,7 @@ __device__ __forceinline__ void sel_block_find(const uint32_t* hist, int nb, int
 // the exact selection over the slices in global memory.  Either way the result
 // equals a full stable sort by (score desc, position asc).
 template <int CS>
-// CS = 16 runs only for few long rows (one CTA per SM): it may use twice the
-// registers, for twice the loads in flight in the collect pass.
-__global__ void __launch_bounds__(kSelThreads, CS == 16 ? 1 : 2) k_select_sampled(const __grid_constant__ SelectArgs a,
+__global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_constant__ SelectArgs a,
                                                                 int32_t* count) {
   grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ uint4 ss_dyn[];
@@ -580,7 +578,7 @@ __global__ void __launch_bounds__(kSelThreads, CS == 16 ? 1 : 2) k_select_sample
 
   // ---- 2. collect every key >= tau of the slice (unordered)
   {
-    constexpr int kBatch = CS == 16 ? 16 : 8;
+    constexpr int kBatch = 8;
     const int64_t len4 = vec ? (len & ~int64_t(3)) : 0;
     auto keep = [&](uint32_t u, int64_t o) {
       if (u >= tau) {

@@ -17,10 +17,12 @@
 // and the cluster merges the partials through distributed shared memory, CTA c
 // finishing the heads h = c mod kSpCluster after a single cluster barrier.  No
 // workspace, no global round trip, no atomics.
-// Many rows (a chunk of queries, bf16): one CTA per row, each warp streaming
-// its own slices through a private ring with 16-byte cp.async copies; there
-// the rows mostly come from L2, where per-lane copies keep up better than one
-// TMA request per 256-byte row.
+// Many rows (a chunk of queries, bf16): one CTA per row, the rows taken KV
+// head by KV head (the CTAs resident at once then share one head's part of the
+// cache, which mostly stays in L2), each warp streaming its own slices through
+// a private ring with 16-byte cp.async copies; there the rows mostly come from
+// L2, where per-lane copies keep up better than one TMA request per 256-byte
+// row.
 //
 // The same kernels run the sliding-window layer of the Hybrid SWA baseline
 // ("Xiaomi Releases HySparse2, Targeting Long-Horizon Reasoning for Agents",
@@ -72,11 +74,21 @@ struct SpRow {
   int64_t r, qi, kv_start, t, pos0;
   int g, cnt, j0, n;
 };
-__device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int cs) {
+// group_major: CTA (cluster) i takes row (query i % total_q, KV head i /
+// total_q), so the CTAs that run at the same time gather from one KV head's
+// part of the cache (it then mostly stays in L2); otherwise row i.
+__device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int cs, bool group_major = false) {
   SpRow s;
-  s.r = blockIdx.x / cs;
-  s.qi = s.r / a.Hkv;
-  s.g = (int)(s.r % a.Hkv);
+  const int64_t i = blockIdx.x / cs;
+  if (group_major) {
+    s.qi = i % a.total_q;
+    s.g = (int)(i / a.total_q);
+    s.r = s.qi * a.Hkv + s.g;
+  } else {
+    s.r = i;
+    s.qi = s.r / a.Hkv;
+    s.g = (int)(s.r % a.Hkv);
+  }
   const QueryRow q = query_row(a.qoff, a.kvoff, a.B, s.qi);
   s.kv_start = q.kv_start;
   s.t = q.t;
@@ -394,7 +406,7 @@ __global__ void __launch_bounds__(32 * kSrWarps) k_sparse_rows_bf16(const __grid
   grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ __align__(128) uint8_t sr_smem[];
   __shared__ float wm[kSrWarps * 8], wl[kSrWarps * 8];
-  const SpRow s = sparse_row(a, 0, 1);  // the whole row (one CTA, rank 0 of 1)
+  const SpRow s = sparse_row(a, 0, 1, true);  // the whole row (one CTA), KV head by KV head
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bf16* K = static_cast<const bf16*>(a.K);
   const bf16* V = static_cast<const bf16*>(a.V);
