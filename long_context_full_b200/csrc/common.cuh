@@ -49,18 +49,23 @@ __device__ __forceinline__ QueryRow query_row(const int64_t* qoff, const int64_t
   return r;
 }
 
+// floor(a / b) for 0 <= a < 2^53 and 0 < b < 2^31, by one fp64 division.  Exact:
+// a non-integer quotient q (< 2^53 / b) lies at least 1/b below the next
+// integer, more than the division's rounding error q * 2^-53.  (The keys and
+// CTA counts here keep a below 2^48.)
+__device__ __forceinline__ int64_t floor_div_f64(int64_t a, int64_t b) {
+  return (int64_t)floor((double)a / (double)b);
+}
+
 // Balanced split of W keys over P CTAs: CTA p owns keys [W*p/P, W*(p+1)/P).
 __device__ __forceinline__ int64_t split_lo(int64_t W, int P, int p) {
-  return (W * (int64_t)p) / (int64_t)P;
+  return floor_div_f64(W * (int64_t)p, P);
 }
-// The CTA that owns key x (0 <= x < W): the largest p with split_lo(p) <= x.
+// The CTA that owns key x (0 <= x < W): the largest p with split_lo(p) <= x,
+// i.e. W p < (x + 1) P, p = floor(((x + 1) P - 1) / W), within [0, P - 1].
 __device__ __forceinline__ int split_owner(int64_t W, int P, int64_t x) {
-  int lo = 0, hi = P - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (split_lo(W, P, mid) <= x) lo = mid; else hi = mid - 1;
-  }
-  return lo;
+  const int64_t q = floor_div_f64((x + 1) * (int64_t)P - 1, W);
+  return (int)(q < 0 ? 0 : (q > P - 1 ? P - 1 : q));
 }
 
 // Order-preserving 32-bit key of a float score: larger score -> larger key,

@@ -76,6 +76,24 @@ __device__ __forceinline__ void for_each_piece(const DecodeArgs& a, int p, F f) 
   }
 }
 
+// A CTA whose key range is empty (more CTAs than keys) writes, for the
+// sequence holding its start, partials that carry nothing (m = -inf, l = 0,
+// O = 0), so that the merge of that sequence's CTAs [split_owner(kb),
+// split_owner(ke - 1)] - which contains such a CTA only strictly inside a
+// sequence - needs no check.  Warp ``w`` of the CTA writes its own slot.
+__device__ __forceinline__ void empty_range_partials(const DecodeArgs& a, int p, int g, int w) {
+  const int64_t lo = split_lo(a.total_kv, a.P, p), hi = split_lo(a.total_kv, a.P, p + 1);
+  if (lo < hi || lo >= a.total_kv) return;
+  const int b = last_le(a.kvoff, a.B, lo);
+  const int64_t base = ((((int64_t)p + b) * a.Hkv + g) * kDecWarps + w) * a.G;
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < a.G * kD; i += 32) a.po[base * kD + i] = 0.f;
+  if (lane < a.G) {
+    a.pm[base + lane] = -INFINITY;
+    a.pl[base + lane] = 0.f;
+  }
+}
+
 // ----------------------------------------------------------------------------
 // bf16 split-context pass on the tensor cores (mma.sync m16n8k16).
 // Per warp and 16-key slice of a tile:  S^T[16 keys x 8 heads] = K Q^T, then
@@ -145,6 +163,7 @@ __device__ __forceinline__ bool decode_stream_bf16(const CUtensorMap* tmK, const
   }
 
   // -------------------------------------------------------------- consumers
+  empty_range_partials(a, p, g, warp);
   const bf16* Q = static_cast<const bf16*>(a.Q);
   const uint64_t keep = policy_evict_last();
   const int r = lane >> 2, qd = lane & 3;
@@ -348,6 +367,7 @@ __global__ void __launch_bounds__(32 * kDecWarps) k_decode_f32(const __grid_cons
   const float* Q = static_cast<const float*>(a.Q);
   const float* K = static_cast<const float*>(a.K);
   const float* V = static_cast<const float*>(a.V);
+  empty_range_partials(a, p, g, warp);
   for_each_piece(a, p, [&](int b, int64_t s, int64_t e, int64_t q0) {
     float4 q[GP];
     float m[GP], l[GP];
@@ -434,18 +454,14 @@ __global__ void __launch_bounds__(kCombThreads) k_decode_combine(const __grid_co
     pf = split_owner(W, a.P, kb);
     np = (split_owner(W, a.P, ke - 1) - pf + 1) * a.nw;
   }
-  // partial i = (CTA pf + i / nw, warp i % nw)
+  // partial i = (CTA pf + i / nw, warp i % nw); CTAs with an empty range wrote
+  // neutral partials (empty_range_partials)
   auto pidx = [&](int i) -> int64_t {
     return (((int64_t)(pf + i / a.nw + b) * a.Hkv + g) * kDecWarps + (i % a.nw)) * a.G + hl;
   };
-  auto valid = [&](int i) {  // CTAs with an empty range wrote nothing
-    const int p = pf + i / a.nw;
-    return split_lo(W, a.P, p) < split_lo(W, a.P, p + 1);
-  };
   // ---- the maximum over the partials
   float M = -INFINITY;
-  for (int i = threadIdx.x; i < np; i += kCombThreads)
-    if (valid(i)) M = fmaxf(M, __ldcg(a.pm + pidx(i)));
+  for (int i = threadIdx.x; i < np; i += kCombThreads) M = fmaxf(M, __ldcg(a.pm + pidx(i)));
   M = warp_max(M);
   if (lane == 0) red[warp] = M;
   __syncthreads();
@@ -459,12 +475,9 @@ __global__ void __launch_bounds__(kCombThreads) k_decode_combine(const __grid_co
   for (int c0 = 0; c0 < np; c0 += kCombCap) {
     const int n = min(kCombCap, np - c0);
     for (int i = threadIdx.x; i < n; i += kCombThreads) {
-      float w = 0.f;
-      if (valid(c0 + i)) {
-        const int64_t pi = pidx(c0 + i);
-        w = exp_shift(__ldcg(a.pm + pi), M);
-        L = fmaf(w, __ldcg(a.pl + pi), L);
-      }
+      const int64_t pi = pidx(c0 + i);
+      const float w = exp_shift(__ldcg(a.pm + pi), M);
+      L = fmaf(w, __ldcg(a.pl + pi), L);
       wsh[i] = w;
     }
     __syncthreads();
@@ -585,10 +598,9 @@ __device__ __forceinline__ void seq_owners(const DecodeArgs& a, int b, int* pf, 
 }
 
 // Index of partial i (= CTA pf + i / nw, warp i % nw) of (sequence b, KV head
-// g, head hl); -1 for a CTA with an empty range (it wrote nothing).
+// g, head hl).  A CTA with an empty key range wrote a neutral partial.
 __device__ __forceinline__ int64_t partial_at(const DecodeArgs& a, int b, int g, int hl, int pf, int i) {
   const int p = pf + i / a.nw;
-  if (split_lo(a.total_kv, a.P, p) >= split_lo(a.total_kv, a.P, p + 1)) return -1;
   return (((int64_t)(p + b) * a.Hkv + g) * kDecWarps + (i % a.nw)) * a.G + hl;
 }
 
@@ -604,16 +616,13 @@ __device__ __forceinline__ void head_stats(const DecodeArgs& a, int b, int g, in
     const int i = u * 32 + lane;
     mv[u] = -INFINITY;
     lv[u] = 0.f;
-    const int64_t pi = i < np ? partial_at(a, b, g, hl, pf, i) : -1;
-    if (pi >= 0) {
+    if (i < np) {
+      const int64_t pi = partial_at(a, b, g, hl, pf, i);
       mv[u] = __ldcg(a.pm + pi);
       lv[u] = __ldcg(a.pl + pi);
     }
   }
-  for (int i = R * 32 + lane; i < np; i += 32) {
-    const int64_t pi = partial_at(a, b, g, hl, pf, i);
-    if (pi >= 0) M = fmaxf(M, __ldcg(a.pm + pi));
-  }
+  for (int i = R * 32 + lane; i < np; i += 32) M = fmaxf(M, __ldcg(a.pm + partial_at(a, b, g, hl, pf, i)));
 #pragma unroll
   for (int u = 0; u < R; ++u) M = fmaxf(M, mv[u]);
   M = warp_max(M);
@@ -622,7 +631,7 @@ __device__ __forceinline__ void head_stats(const DecodeArgs& a, int b, int g, in
   for (int u = 0; u < R; ++u) L = fmaf(exp_shift(mv[u], M), lv[u], L);
   for (int i = R * 32 + lane; i < np; i += 32) {
     const int64_t pi = partial_at(a, b, g, hl, pf, i);
-    if (pi >= 0) L = fmaf(exp_shift(__ldcg(a.pm + pi), M), __ldcg(a.pl + pi), L);
+    L = fmaf(exp_shift(__ldcg(a.pm + pi), M), __ldcg(a.pl + pi), L);
   }
   *Mo = M;
   *Lo = warp_sum(L);
@@ -635,9 +644,8 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_co
   grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ __align__(128) float fring[];
   __shared__ __align__(8) uint64_t full_bar[kFinStages], empty_bar[kFinStages];
-  __shared__ float wsh[kCombCap];
   __shared__ __align__(16) float4 osh[kFinWarps][32];
-  __shared__ float red[kFinWarps];
+  __shared__ float red[kFinWarps], redm[kFinWarps];
   __shared__ float cm[16], cl[16];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.x, g = blockIdx.y;
@@ -710,67 +718,58 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_co
       int pf, pn;
       seq_owners(a, b, &pf, &pn);
       const int np = pn * a.nw;
-      float M = -INFINITY;
-      for (int i = threadIdx.x; i < np; i += NC) {
-        const int64_t pi = partial_at(a, b, gi, hl, pf, i);
-        if (pi >= 0) M = fmaxf(M, __ldcg(a.pm + pi));
-      }
-      M = warp_max(M);
-      if (lane == 0) red[warp] = M;
-      named_barrier_sync(1, NC);
-      M = red[0];
-#pragma unroll
-      for (int w = 1; w < kFinWarps; ++w) M = fmaxf(M, red[w]);
-      float L = 0.f;
+      // warp w merges partials w, w + 8, ... with a running maximum, U of them
+      // loaded at once (m, l and its 16 bytes of O per lane), then warp 0
+      // merges the eight warps' results
+      float M = -INFINITY, L = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c0 = 0; c0 < np; c0 += kCombCap) {
-        const int n = min(kCombCap, np - c0);
-        named_barrier_sync(1, NC);  // red[] / wsh[] of the step before are read
-        for (int i = threadIdx.x; i < n; i += NC) {
-          float w = 0.f;
-          const int64_t pi = partial_at(a, b, gi, hl, pf, c0 + i);
-          if (pi >= 0) {
-            w = exp_shift(__ldcg(a.pm + pi), M);
-            L = fmaf(w, __ldcg(a.pl + pi), L);
+      constexpr int U = 8;
+      for (int i0 = warp; i0 < np; i0 += kFinWarps * U) {
+        float mv[U], lv[U];
+        float4 ov[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int i = i0 + u * kFinWarps;
+          mv[u] = -INFINITY;
+          lv[u] = 0.f;
+          ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < np) {
+            const int64_t pi = partial_at(a, b, gi, hl, pf, i);
+            mv[u] = __ldcg(a.pm + pi);
+            lv[u] = __ldcg(a.pl + pi);
+            ov[u] = __ldcg(reinterpret_cast<const float4*>(a.po + pi * kD) + lane);
           }
-          wsh[i] = w;
         }
-        named_barrier_sync(1, NC);
-        constexpr int U = 4;
-        for (int i0 = warp; i0 < n; i0 += kFinWarps * U) {
-          float4 o[U];
-          float wt[U];
 #pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int i = i0 + u * kFinWarps;
-            wt[u] = i < n ? wsh[i] : 0.f;
-            const int pp = pf + (c0 + i) / a.nw;
-            const int64_t pi = (((int64_t)(pp + b) * a.Hkv + gi) * kDecWarps + ((c0 + i) % a.nw)) * G + hl;
-            o[u] = wt[u] != 0.f ? __ldcg(reinterpret_cast<const float4*>(a.po + pi * kD) + lane)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            acc.x = fmaf(wt[u], o[u].x, acc.x);
-            acc.y = fmaf(wt[u], o[u].y, acc.y);
-            acc.z = fmaf(wt[u], o[u].z, acc.z);
-            acc.w = fmaf(wt[u], o[u].w, acc.w);
-          }
+        for (int u = 0; u < U; ++u) {
+          const float Mn = fmaxf(M, mv[u]);
+          const float so = exp_shift(M, Mn), w = exp_shift(mv[u], Mn);
+          L = fmaf(L, so, w * lv[u]);
+          acc.x = fmaf(acc.x, so, w * ov[u].x);
+          acc.y = fmaf(acc.y, so, w * ov[u].y);
+          acc.z = fmaf(acc.z, so, w * ov[u].z);
+          acc.w = fmaf(acc.w, so, w * ov[u].w);
+          M = Mn;
         }
       }
-      L = warp_sum(L);
       osh[warp][lane] = acc;
-      named_barrier_sync(1, NC);
-      if (lane == 0) red[warp] = L;
+      if (lane == 0) {
+        red[warp] = L;
+        redm[warp] = M;
+      }
       named_barrier_sync(1, NC);
       if (warp == 0) {
+        float Mt = redm[0];
+#pragma unroll
+        for (int w = 1; w < kFinWarps; ++w) Mt = fmaxf(Mt, redm[w]);
         float Lt = 0.f;
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < kFinWarps; ++w) {
-          Lt += red[w];
+          const float f = exp_shift(redm[w], Mt);
+          Lt = fmaf(f, red[w], Lt);
           const float4 v = osh[w][lane];
-          o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+          o.x = fmaf(f, v.x, o.x); o.y = fmaf(f, v.y, o.y); o.z = fmaf(f, v.z, o.z); o.w = fmaf(f, v.w, o.w);
         }
         const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
         OT* dst = O + (q0 * a.Hq + h) * kD + lane * 4;
