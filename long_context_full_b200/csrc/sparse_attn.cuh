@@ -74,10 +74,18 @@ struct SpRow {
   int64_t r, qi, kv_start, t, pos0;
   int g, cnt, j0, n;
 };
+// The share of a CTA of a cs-CTA cluster: list entries [rank * per, ...),
+// per = ceil(cnt / cs) rounded up to 16.
+__device__ __forceinline__ int sparse_share(int cnt, int cs) { return ((cnt + cs - 1) / cs + 15) / 16 * 16; }
+
 // group_major: CTA (cluster) i takes row (query i % total_q, KV head i /
 // total_q), so the CTAs that run at the same time gather from one KV head's
 // part of the cache (it then mostly stays in L2); otherwise row i.
-__device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int cs, bool group_major = false) {
+// block_search: the whole CTA calls it, and finds the query's sequence with one
+// round of loads (one offset per thread and a barrier count) when B fits the
+// CTA, instead of a binary search of dependent loads.
+__device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int cs, bool group_major = false,
+                                            bool block_search = false) {
   SpRow s;
   const int64_t i = blockIdx.x / cs;
   if (group_major) {
@@ -89,7 +97,21 @@ __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int c
     s.qi = s.r / a.Hkv;
     s.g = (int)(s.r % a.Hkv);
   }
-  const QueryRow q = query_row(a.qoff, a.kvoff, a.B, s.qi);
+  const int cnt_in = a.window > 0 ? 0 : __ldg(a.count + s.r);  // independent of the search
+  QueryRow q;
+  if (block_search && a.B <= (int)blockDim.x) {
+    // the last b with qoff[b] <= qi: the number of b' in [1, B] with
+    // qoff[b'] <= qi (offsets ascending, qoff[0] = 0), at most B - 1
+    const int b1 = (int)threadIdx.x + 1;
+    const int c = __syncthreads_count(b1 <= a.B && __ldg(a.qoff + b1) <= s.qi);
+    q.b = c < a.B ? c : a.B - 1;
+    const int64_t q0 = __ldg(a.qoff + q.b), q1 = __ldg(a.qoff + q.b + 1);
+    q.kv_start = __ldg(a.kvoff + q.b);
+    q.kv_len = __ldg(a.kvoff + q.b + 1) - q.kv_start;
+    q.t = q.kv_len - (q1 - q0) + (s.qi - q0);
+  } else {
+    q = query_row(a.qoff, a.kvoff, a.B, s.qi);
+  }
   s.kv_start = q.kv_start;
   s.t = q.t;
   s.pos0 = a.pos0 ? __ldg(a.pos0 + q.b) : 0;
@@ -97,25 +119,22 @@ __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int c
   if (a.window > 0) {  // sliding window: the last min(window, t + 1) positions
     cnt = (int)(s.t + 1 < 0 ? 0 : (s.t + 1 < a.window ? s.t + 1 : a.window));
   } else {
-    cnt = __ldg(a.count + s.r);
+    cnt = cnt_in;
     if (cnt < 0 || cnt > a.idx_stride) {
       if (threadIdx.x == 0 && rank == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
       cnt = cnt < 0 ? 0 : a.idx_stride;
     }
   }
   s.cnt = cnt;
-  int per = (cnt + cs - 1) / cs;
-  per = (per + 15) / 16 * 16;
+  const int per = sparse_share(cnt, cs);
   s.j0 = rank * per;
   s.n = cnt - s.j0 < 0 ? 0 : (cnt - s.j0 < per ? cnt - s.j0 : per);
   return s;
 }
 
-// Cache position of list entry i of the CTA's share (window mode: the i-th
-// position of the window), or -1 (recorded) if outside 0..t.
-__device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& s, int i,
-                                              bool record) {
-  int64_t pos = a.window > 0 ? s.t - s.cnt + 1 + s.j0 + i : __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
+// Cache position of a list entry's value ``pos`` (index mode), or -1
+// (recorded) if outside 0..t.
+__device__ __forceinline__ int64_t sparse_checked(const SparseArgs& a, const SpRow& s, int64_t pos, bool record) {
   if (a.pos0) {  // a global position: another rank's row is skipped, not an error
     pos -= s.pos0;
     if (pos < 0 || pos > s.t) return -1;
@@ -125,6 +144,15 @@ __device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& 
     return -1;
   }
   return pos;
+}
+
+// Cache position of list entry i of the CTA's share (window mode: the i-th
+// position of the window), or -1 (recorded) if outside 0..t.
+__device__ __forceinline__ int64_t sparse_pos(const SparseArgs& a, const SpRow& s, int i,
+                                              bool record) {
+  const int64_t pos =
+      a.window > 0 ? s.t - s.cnt + 1 + s.j0 + i : __ldg(a.idx + s.r * a.idx_stride + s.j0 + i);
+  return sparse_checked(a, s, pos, record);
 }
 
 // Partials received by the CTA that finishes a head: one slot per source CTA
@@ -247,7 +275,20 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
     mbar_init(&gbar[1], 1);
     fence_mbar_init();
   }
-  const SpRow s = sparse_row(a, rank, cs);
+  // the list entries of this CTA's share when the list is full (count ==
+  // idx_stride, the usual case), loaded before the count is known
+  int64_t spec[2] = {-1, -1};
+  const int per_full = sparse_share(a.idx_stride, cs);
+  if (a.window == 0) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = rank * per_full + (int)threadIdx.x + u * (int)blockDim.x;
+      if ((int)threadIdx.x + u * (int)blockDim.x < per_full && e < a.idx_stride)
+        spec[u] = __ldg(a.idx + (int64_t)(blockIdx.x / cs) * a.idx_stride + e);
+    }
+  }
+  const SpRow s = sparse_row(a, rank, cs, false, true);
+  const bool spec_ok = a.window == 0 && s.j0 == rank * per_full && per_full <= 2 * (int)blockDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // staged rows: K and V, each as two [kSpPiece][128 B] halves (columns 0-63,
   // 64-127) in the 128-byte swizzle of the tensor maps, bases 1024-aligned
@@ -282,8 +323,13 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
     const int pn = s.n - p0 < kSpPiece ? s.n - p0 : kSpPiece;
     const int ntile = (pn + 15) / 16;
     // the piece's cache rows (-1: past the list or invalid), read once
-    for (int row = threadIdx.x; row < ntile * 16; row += blockDim.x)
-      spos[row] = row < pn ? sparse_pos(a, s, p0 + row, true) : -1;
+    for (int row = threadIdx.x, u = 0; row < ntile * 16; row += blockDim.x, ++u) {
+      int64_t pos = -1;
+      if (row < pn)
+        pos = (spec_ok && p0 == 0 && u < 2) ? sparse_checked(a, s, u == 0 ? spec[0] : spec[1], true)
+                                              : sparse_pos(a, s, p0 + row, true);
+      spos[row] = pos;
+    }
     __syncthreads();
     // gather: one TMA gather4 per 4 rows and per 64-column half of K and of V
     // (rows past pn or with an invalid index load a row of the sequence that
