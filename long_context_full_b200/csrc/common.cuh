@@ -49,6 +49,25 @@ __device__ __forceinline__ QueryRow query_row(const int64_t* qoff, const int64_t
   return r;
 }
 
+// query_row for a whole CTA (every thread calls it, with the same qi): the
+// sequence is the number of b' in [1, B] with qoff[b'] <= qi (offsets
+// ascending from qoff[0] = 0), at most B - 1, found with one load per thread
+// and a barrier count instead of a binary search of dependent loads.  Falls
+// back to query_row when B exceeds the CTA.
+__device__ __forceinline__ QueryRow query_row_block(const int64_t* qoff, const int64_t* kvoff, int B,
+                                                    int64_t qi) {
+  if (B > (int)blockDim.x) return query_row(qoff, kvoff, B, qi);
+  const int b1 = (int)threadIdx.x + 1;
+  const int c = __syncthreads_count(b1 <= B && __ldg(qoff + b1) <= qi);
+  QueryRow r;
+  r.b = c < B ? c : B - 1;
+  const int64_t q0 = __ldg(qoff + r.b), q1 = __ldg(qoff + r.b + 1);
+  r.kv_start = __ldg(kvoff + r.b);
+  r.kv_len = __ldg(kvoff + r.b + 1) - r.kv_start;
+  r.t = r.kv_len - (q1 - q0) + (qi - q0);
+  return r;
+}
+
 // floor(a / b) for 0 <= a < 2^53 and 0 < b < 2^31, by one fp64 division.  Exact:
 // a non-integer quotient q (< 2^53 / b) lies at least 1/b below the next
 // integer, more than the division's rounding error q * 2^-53.  (The keys and

@@ -849,6 +849,16 @@ __global__ void __launch_bounds__(kFinThreads) k_finalize_scores(const __grid_co
             out[j0 + i] = sc;
           }
         }
+        // The chunk's logits, written by this call's pass, are dead once copied
+        // in: drop the L2 lines wholly inside it (no other chunk reads them), so
+        // those still held in L2 are never written back to DRAM.  (With ml_in
+        // the logits belong to the caller's workspace and are left alone.)
+        if (!ml_in) {
+          const uintptr_t lo = (reinterpret_cast<uintptr_t>(lg + j0 * Gp) + 127) & ~uintptr_t(127);
+          const uintptr_t hi = reinterpret_cast<uintptr_t>(lg + top * Gp) & ~uintptr_t(127);
+          for (uintptr_t l = lo + (uintptr_t)threadIdx.x * 128; l < hi; l += (uintptr_t)NC * 128)
+            discard_l2(reinterpret_cast<const void*>(l));
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[stage]);

@@ -93,6 +93,12 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
+// Drops the 128-byte L2 line at p (global memory, 128-byte aligned) without
+// writing it back: the line's contents are undefined until written again.
+// For scratch data that is dead once read.
+__device__ __forceinline__ void discard_l2(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
 // Stores with an L2 eviction-priority hint.
 __device__ __forceinline__ void st_hint_f2(float* p, float a, float b, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(a), "f"(b),

@@ -69,8 +69,11 @@ struct SelState {
 
 // Number of candidates of a row: positions [0, t-window] (token rows) or the
 // blocks holding at least one of them (block rows).  Sets *t.
-__device__ __forceinline__ int64_t sel_row_candidates(const SelectArgs& a, int64_t r, int64_t* t) {
-  const QueryRow q = query_row(a.qoff, a.kvoff, a.B, r / a.Hkv);
+// block_search: the whole CTA calls it (query_row_block).
+__device__ __forceinline__ int64_t sel_row_candidates(const SelectArgs& a, int64_t r, int64_t* t,
+                                                      bool block_search = false) {
+  const QueryRow q = block_search ? query_row_block(a.qoff, a.kvoff, a.B, r / a.Hkv)
+                                  : query_row(a.qoff, a.kvoff, a.B, r / a.Hkv);
   *t = q.t;
   int64_t nc = q.t - a.window + 1;
   if (nc < 0) nc = 0;
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_
   const float* row = a.data + r * a.stride + j0;
   const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15) == 0);
   int64_t t;
-  int64_t nc = sel_row_candidates(a, r, &t);
+  int64_t nc = sel_row_candidates(a, r, &t, true);
   if (nc > (int64_t)CS * S) {  // longer than the host's maximum
     if (threadIdx.x == 0) record_error(a.err, HS2_ERR_DEVICE_INPUT);
     nc = 0;

@@ -81,9 +81,8 @@ __device__ __forceinline__ int sparse_share(int cnt, int cs) { return ((cnt + cs
 // group_major: CTA (cluster) i takes row (query i % total_q, KV head i /
 // total_q), so the CTAs that run at the same time gather from one KV head's
 // part of the cache (it then mostly stays in L2); otherwise row i.
-// block_search: the whole CTA calls it, and finds the query's sequence with one
-// round of loads (one offset per thread and a barrier count) when B fits the
-// CTA, instead of a binary search of dependent loads.
+// block_search: the whole CTA calls it and finds the query's sequence with
+// query_row_block.
 __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int cs, bool group_major = false,
                                             bool block_search = false) {
   SpRow s;
@@ -98,20 +97,8 @@ __device__ __forceinline__ SpRow sparse_row(const SparseArgs& a, int rank, int c
     s.g = (int)(s.r % a.Hkv);
   }
   const int cnt_in = a.window > 0 ? 0 : __ldg(a.count + s.r);  // independent of the search
-  QueryRow q;
-  if (block_search && a.B <= (int)blockDim.x) {
-    // the last b with qoff[b] <= qi: the number of b' in [1, B] with
-    // qoff[b'] <= qi (offsets ascending, qoff[0] = 0), at most B - 1
-    const int b1 = (int)threadIdx.x + 1;
-    const int c = __syncthreads_count(b1 <= a.B && __ldg(a.qoff + b1) <= s.qi);
-    q.b = c < a.B ? c : a.B - 1;
-    const int64_t q0 = __ldg(a.qoff + q.b), q1 = __ldg(a.qoff + q.b + 1);
-    q.kv_start = __ldg(a.kvoff + q.b);
-    q.kv_len = __ldg(a.kvoff + q.b + 1) - q.kv_start;
-    q.t = q.kv_len - (q1 - q0) + (s.qi - q0);
-  } else {
-    q = query_row(a.qoff, a.kvoff, a.B, s.qi);
-  }
+  const QueryRow q = block_search ? query_row_block(a.qoff, a.kvoff, a.B, s.qi)
+                                  : query_row(a.qoff, a.kvoff, a.B, s.qi);
   s.kv_start = q.kv_start;
   s.t = q.t;
   s.pos0 = a.pos0 ? __ldg(a.pos0 + q.b) : 0;
