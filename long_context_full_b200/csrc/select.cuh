@@ -37,6 +37,16 @@ constexpr int kSelChunkAlign = 128 * kSelWarps;  // slices are multiples of this
 constexpr int kSsCap = 8192;       // sampled kernel: candidates (or samples) one CTA holds
 constexpr int kSsSortMax = 2048;   // sampled kernel: largest k
 constexpr int kSsMinRho = 16;      // sampled kernel: at most one key in 16 is sampled
+constexpr int kSsBcast = 256;      // sampled kernel: keys of the threshold's 22-bit prefix sent to every CTA
+
+// Adds v to the 32-bit word at ``p`` (this CTA's shared memory) in CTA
+// ``cta`` of the cluster, without waiting for a result; the next cluster
+// barrier makes it visible there.
+__device__ __forceinline__ void cluster_red_add(const uint32_t* p, int cta, uint32_t v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(cta));
+  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
+}
 
 struct SelectArgs {
   const float* data;   // rows of values to select from
@@ -469,20 +479,223 @@ __device__ __forceinline__ void sel_block_find(const uint32_t* hist, int nb, int
   __syncthreads();
 }
 
+// Writes the nsel distinct positions sel[0, nsel), all in [lo, lo + span), to
+// out[0, nsel) in ascending order: a counting sort over kSelBins position
+// bins, then an insertion sort of the (few) positions of each bin.  tmp holds
+// nsel ints of scratch.  All threads of the CTA call it.
+template <int CS>
+__device__ void sel_write_ordered(SelState<CS>& st, const int32_t* sel, int nsel, int64_t lo,
+                                  int64_t span, int32_t* tmp, int32_t* out) {
+  int sh = 0;
+  while (((span - 1) >> sh) >= kSelBins) ++sh;
+  auto bin_of = [&](int32_t v) { return (int)(((int64_t)v - lo) >> sh); };
+  for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) st.h[i] = 0u;
+  __syncthreads();
+  for (int e = threadIdx.x; e < nsel; e += kSelThreads) atomicAdd(&st.h[bin_of(sel[e])], 1u);
+  __syncthreads();
+  {
+    constexpr int E = kSelBins / kSelThreads;  // bins per thread, in order
+    uint32_t c[E];
+    int mine = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      c[e] = st.h[threadIdx.x * E + e];
+      mine += (int)c[e];
+    }
+    int tot;
+    int run = block_exclusive_scan(mine, st.wgt, &tot);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      st.h[threadIdx.x * E + e] = (uint32_t)run;  // start of the bin
+      run += (int)c[e];
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < nsel; e += kSelThreads) {
+    const int32_t v = sel[e];
+    tmp[atomicAdd(&st.h[bin_of(v)], 1u)] = v;  // afterwards st.h[b] = end of bin b
+  }
+  __syncthreads();
+  {
+    constexpr int E = kSelBins / kSelThreads;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int bin = threadIdx.x * E + e;
+      const int b0 = bin ? (int)st.h[bin - 1] : 0, b1 = (int)st.h[bin];
+      for (int i = b0 + 1; i < b1; ++i) {
+        const int32_t v = tmp[i];
+        int j = i - 1;
+        while (j >= b0 && tmp[j] > v) {
+          tmp[j + 1] = tmp[j];
+          --j;
+        }
+        tmp[j + 1] = v;
+      }
+      for (int i = b0; i < b1; ++i) out[i] = tmp[i];
+    }
+  }
+}
+
+// Cluster-wide state of the gather-free finish of a sampled row (CS > 1).
+template <int CS>
+struct SelFinish {
+  uint32_t hs[kSelBins];  // the cluster's histogram of the sampled keys' top 11 bits
+  uint32_t h1[kSelBins];  // the cluster's histogram of the kept keys' top 11 bits
+  uint32_t h2[kSelBins];  // the cluster's histogram of bits 10-20 of the kept keys of bin d1
+  uint64_t bc[kSsBcast];  // the cluster's kept keys of the 22-bit prefix (d1, d2), with positions
+  int nbc;                // entries in bc
+  int base[CS];           // where this CTA's prefix keys go in CTA c's bc
+  int cgt[CS];            // per CTA: its kept keys above bin d1
+  int cgt2[CS];           // per CTA: its kept keys of bin d1 above sub-bin d2
+  int csel[CS];           // per CTA: its keys of (d1, d2) taken
+};
+
+// The end of a sampled row on a cluster without gathering the kept keys on
+// one CTA.  On entry every CTA holds its kept keys (all >= tau) in cand[0, n)
+// and fin.h1 the cluster's histogram of their top 11 bits (each CTA added its
+// own to every CTA's copy before the last cluster barrier).
+//  a. d1 = the bin of the k-th largest kept key, r1 its rank inside the bin;
+//  b. each CTA adds the histogram of bits 10-20 of its keys of bin d1 to every
+//     CTA's h2 and sends its count of keys above bin d1; a cluster barrier;
+//     d2 = the sub-bin of the r1-th largest key of bin d1, r2 its rank there;
+//  c. each CTA sends its keys of the prefix (d1, d2) -- the threshold key, its
+//     ties and near-ties: few -- with their positions to every CTA, and its
+//     count of keys above the prefix; a cluster barrier;
+//  d. every CTA ranks the prefix's keys by (key desc, position asc) and takes
+//     the r2 first; each CTA writes its selected positions (every key above
+//     the prefix and the taken ones of its slice) in ascending order after
+//     those of the CTAs before it, whose slices hold the lower positions.
+// The selection is the same as the gathering path's.  Returns false, with
+// every CTA alike and the kept keys untouched, when more than kSsBcast keys
+// share the prefix; the caller then takes the gathering path.
+template <int CS>
+__device__ bool sel_cluster_finish(cg::cluster_group& cl, SelState<CS>& st, SelFinish<CS>& fin,
+                                   const SelectArgs& a, uint64_t* cand, int n, int32_t* sel,
+                                   int rank, int64_t S, int32_t* out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < CS) fin.csel[threadIdx.x] = 0;
+  if (threadIdx.x == 0) st.nsel = 0;
+  // a.
+  sel_block_find(fin.h1, kSelBins, a.k, st.wgt, &st.digit, &st.krem);
+  const uint32_t d1 = st.digit;
+  const int r1 = st.krem;
+  // b.
+  for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) st.h[i] = 0u;
+  __syncthreads();
+  int gt = 0;
+  for (int base = warp * 32; base < n; base += kSelThreads) {
+    const int i = base + lane;
+    const uint32_t u = i < n ? (uint32_t)cand[i] : 0u;
+    gt += (i < n && (u >> 21) > d1) ? 1 : 0;
+    sel_hist_add(st.h, (u >> 10) & 0x7FFu, i < n && (u >> 21) == d1);
+  }
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  if (lane == 0) st.wgt[warp] = gt;
+  __syncthreads();
+  for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) {
+    const uint32_t v = st.h[i];
+    if (v)
+      for (int c = 0; c < CS; ++c) cluster_red_add(&fin.h2[i], c, v);
+  }
+  if (threadIdx.x < CS) {  // thread c sends this CTA's count to CTA c
+    int sum = 0;
+    for (int w = 0; w < kSelWarps; ++w) sum += st.wgt[w];
+    *cl.map_shared_rank(&fin.cgt[rank], (int)threadIdx.x) = sum;
+  }
+  cl.sync();
+  sel_block_find(fin.h2, kSelBins, r1, st.wgt, &st.digit, &st.krem);
+  const uint32_t d2 = st.digit;
+  const int r2 = st.krem;
+  const uint32_t pre = (d1 << 11) | d2;  // the threshold's top 22 bits
+  if ((int)fin.h2[d2] > kSsBcast) return false;  // the same on every CTA
+  // c. (the prefix keys first to a local list: one slot reservation per CTA
+  // of the cluster instead of one per key)
+  uint64_t* lst = reinterpret_cast<uint64_t*>(sel);  // sel is written only after the barrier
+  if (threadIdx.x == 0) st.neq = 0;
+  __syncthreads();
+  int gt2 = 0;
+  for (int i = threadIdx.x; i < n; i += kSelThreads) {
+    const uint64_t cv = cand[i];
+    const uint32_t u22 = (uint32_t)cv >> 10;
+    if (u22 > pre && (u22 >> 11) == d1) ++gt2;
+    if (u22 == pre) {
+      const int slot = atomicAdd(&st.neq, 1);
+      if (slot < kSsBcast) lst[slot] = cv;
+    }
+  }
+  gt2 = __reduce_add_sync(0xffffffffu, gt2);
+  if (lane == 0) st.weq[warp] = gt2;
+  __syncthreads();
+  const int m = st.neq < kSsBcast ? st.neq : kSsBcast;
+  if (threadIdx.x < CS) {
+    int sum = 0;
+    for (int w = 0; w < kSelWarps; ++w) sum += st.weq[w];
+    *cl.map_shared_rank(&fin.cgt2[rank], (int)threadIdx.x) = sum;
+    fin.base[threadIdx.x] = m ? atomicAdd(cl.map_shared_rank(&fin.nbc, (int)threadIdx.x), m) : 0;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < m * CS; j += kSelThreads) {
+    const int c = j / m, i = j - c * m;
+    const int slot = fin.base[c] + i;
+    if (slot < kSsBcast) *cl.map_shared_rank(&fin.bc[slot], c) = lst[i];
+  }
+  cl.sync();  // no CTA reads another's shared memory after this
+  // d.
+  const int nb = fin.nbc < kSsBcast ? fin.nbc : kSsBcast;
+  for (int t = threadIdx.x; t < nb; t += kSelThreads) {
+    const uint64_t me = fin.bc[t];
+    const uint32_t u = (uint32_t)me, p = (uint32_t)(me >> 32);
+    int rk = 0;
+    for (int j = 0; j < nb; ++j) {
+      const uint64_t o = fin.bc[j];
+      const uint32_t uo = (uint32_t)o, po = (uint32_t)(o >> 32);
+      rk += (uo > u || (uo == u && po < p)) ? 1 : 0;
+    }
+    if (rk < r2) {
+      const int c = (int)(p / (uint32_t)S);
+      atomicAdd(&fin.csel[c], 1);
+      if (c == rank) sel[atomicAdd(&st.nsel, 1)] = (int32_t)p;
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += kSelThreads) {
+    const uint64_t cv = cand[i];
+    if (((uint32_t)cv >> 10) > pre) sel[atomicAdd(&st.nsel, 1)] = (int32_t)(cv >> 32);
+  }
+  __syncthreads();
+  int before = 0;
+  for (int c = 0; c < rank; ++c) before += fin.cgt[c] + fin.cgt2[c] + fin.csel[c];
+  const int nown = st.nsel;
+  if (nown <= 160) {  // few (a decode row's share): each one's rank among them by counting
+    for (int t = threadIdx.x; t < nown; t += kSelThreads) {
+      const int32_t p = sel[t];
+      int rk = 0;
+      for (int j = 0; j < nown; ++j) rk += sel[j] < p ? 1 : 0;
+      out[before + rk] = p;
+    }
+  } else {  // the kept keys are no longer read: their buffer is the scratch
+    sel_write_ordered(st, sel, nown, (int64_t)rank * S, S, reinterpret_cast<int32_t*>(cand), out + before);
+  }
+  return true;
+}
+
 // Sample-guided exact selection (k <= kSsSortMax), one cluster of CS CTAs
 // (CS may be 1) per row; CTA c owns the c-th slice of the row's candidates.
 //  1. Sample: one group of four consecutive keys from every 4*rho keys (rho >=
-//     16, at a hashed offset inside the group).  Every CTA sums the cluster's
-//     histograms of the sampled keys' top 11 bits and takes tau = the smallest
-//     key of the bin holding the rs-th largest sample, rs = k/rho plus a margin
-//     of four standard deviations.
+//     16, at a hashed offset inside the group).  Every CTA adds its histogram
+//     of the sampled keys' top 11 bits to every CTA's copy of the cluster's
+//     histogram and takes tau = the smallest key of the bin holding the rs-th
+//     largest sample, rs = k/rho plus a margin of four standard deviations.
 //  2. Collect: one pass over the slice keeps every key >= tau with its
 //     position.  When the cluster holds at least k such keys, the row's k
 //     largest keys are all among them.
-//  3. CTA 0 gathers the kept keys of the cluster, finds the k-th largest key T
-//     and the number kr of keys == T to take by a radix select, keeps every
-//     key > T and the kr lowest-position keys == T, and writes the kept
-//     positions in ascending order (each one's rank among them).
+//  3. Clusters over rows that reach the last CTA's slice: every CTA finds the
+//     threshold from the cluster's histograms of the kept keys and writes its
+//     own share of the result (sel_cluster_finish).  Otherwise, or when too
+//     many keys share the threshold's 22-bit prefix, CTA
+//     0 gathers the kept keys of the cluster, finds the k-th largest key T and
+//     the number kr of keys == T to take by a radix select, keeps every key > T
+//     and the kr lowest-position keys == T, and writes the kept positions in
+//     ascending order.
 // Otherwise (fewer than k kept, or more than one CTA holds) the cluster runs
 // the exact selection over the slices in global memory.  Either way the result
 // equals a full stable sort by (score desc, position asc).
@@ -495,6 +708,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_
   int32_t* sel = reinterpret_cast<int32_t*>(cand + kSsCap);       // selected positions
   __shared__ SelState<CS> st;
   __shared__ int offs[CS + 1];
+  __shared__ SelFinish<CS> fin;
   cg::cluster_group cl = cg::this_cluster();
   const int rank = CS == 1 ? 0 : (int)cl.block_rank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -525,6 +739,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_
 
   // ---- 1. sample (rho depends on the slice size only: the same on every CTA)
   for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) st.h[i] = 0u;
+  if constexpr (CS > 1) {  // the finish's cluster histograms, filled by every CTA later
+    for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) fin.hs[i] = fin.h1[i] = fin.h2[i] = 0u;
+    if (threadIdx.x == 0) fin.nbc = 0;
+  }
   if (threadIdx.x == 0) {
     st.n = 0;
     st.ns = 0;
@@ -562,17 +780,25 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_
     }
   }
   if (threadIdx.x == 0) st.ns = 4 * ngroups;
+  if constexpr (CS > 1) {
+    // this CTA's sample histogram added to every CTA's fin.hs
+    __syncthreads();
+    for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) {
+      const uint32_t v = st.h[i];
+      if (v)
+        for (int c = 0; c < CS; ++c) cluster_red_add(&fin.hs[i], c, v);
+    }
+  }
   csync();
   // tau = the lower edge of the bin holding the rs-th largest sample of the
-  // row.  CS > 1: the cluster's sample histograms are reduce-scattered (CTA c
-  // sums bins [c*own, (c+1)*own) over the cluster) and every CTA finds the
-  // same bin from the totals; a row with fewer than rs samples keeps tau = 0.
+  // row (every CTA finds the same bin in its copy of the cluster's sample
+  // histogram); a row with fewer than rs samples keeps tau = 0.
   const float kr_f = (float)a.k / (float)rho;
   const int rs = (int)ceilf(kr_f + 4.f * sqrtf(kr_f)) + 8;
   uint32_t tau = 0u;
   if constexpr (CS > 1) {
-    const int own = sel_reduce_bins<CS>(cl, st, kSelBins);
-    sel_find_digit<CS>(cl, st, own, rs);
+    if (threadIdx.x == 0) st.digit = 0u;  // kept when the samples are fewer than rs
+    sel_block_find(fin.hs, kSelBins, rs, st.wgt, &st.digit, &st.krem);
     tau = st.digit << 21;
   } else if (st.ns >= rs) {
     sel_block_find(st.h, kSelBins, rs, st.wgt, &st.digit, &st.krem);
@@ -609,6 +835,28 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_
     }
     for (int64_t i = len4 + threadIdx.x; i < len; i += kSelThreads) keep(key_at(i), i);
   }
+  // the gather-free finish when every CTA of the cluster holds part of the
+  // row (a shorter row leaves CTAs idle there: the gathering path lets them
+  // go early)
+  const bool spread = CS > 1 && nc > (int64_t)(CS - 1) * S;
+  if (spread) {
+    // this CTA's histogram of its kept keys' top 11 bits, added to every CTA's
+    // fin.h1
+    __syncthreads();  // st.n is final
+    const int nloc = st.n < kSsCap ? st.n : kSsCap;
+    for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) st.h[i] = 0u;
+    __syncthreads();
+    for (int base = warp * 32; base < nloc; base += kSelThreads) {
+      const int i = base + lane;
+      sel_hist_add(st.h, i < nloc ? (uint32_t)cand[i] >> 21 : 0u, i < nloc);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) {
+      const uint32_t v = st.h[i];
+      if (v)
+        for (int c = 0; c < CS; ++c) cluster_red_add(&fin.h1[i], c, v);
+    }
+  }
   csync();
   int collected = 0, most = 0;
   if (threadIdx.x == 0) offs[0] = 0;
@@ -623,6 +871,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_
     // the sample misled: exact selection over the slices in global memory
     sel_exact<CS>(cl, st, a, row, j0, S, len, false, vec, nullptr, out);
     return;
+  }
+  if (spread) {
+    if (sel_cluster_finish<CS>(cl, st, fin, a, cand, st.n, sel, rank, S, out)) return;
   }
 
   // ---- 3. CTA 0 gathers the cluster's kept keys and finishes the row
@@ -710,56 +961,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select_sampled(const __grid_
   }
   __syncthreads();
   // ascending order by a counting sort over position bins (positions < nc)
-  const int nsel = ngt + kr;
-  int sh = 0;
-  while (((nc - 1) >> sh) >= kSelBins) ++sh;
-  for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) st.h[i] = 0u;
-  __syncthreads();
-  for (int e = threadIdx.x; e < nsel; e += kSelThreads) atomicAdd(&st.h[sel[e] >> sh], 1u);
-  __syncthreads();
-  {
-    constexpr int E = kSelBins / kSelThreads;  // bins per thread, in order
-    uint32_t c[E];
-    int mine = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      c[e] = st.h[threadIdx.x * E + e];
-      mine += (int)c[e];
-    }
-    int tot;
-    int run = block_exclusive_scan(mine, st.wgt, &tot);
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      st.h[threadIdx.x * E + e] = (uint32_t)run;  // start of the bin
-      run += (int)c[e];
-    }
-  }
-  __syncthreads();
-  int32_t* tmp = reinterpret_cast<int32_t*>(cand);  // kept keys are no longer needed
-  for (int e = threadIdx.x; e < nsel; e += kSelThreads) {
-    const int32_t v = sel[e];
-    tmp[atomicAdd(&st.h[v >> sh], 1u)] = v;  // afterwards st.h[b] = end of bin b
-  }
-  __syncthreads();
-  {
-    constexpr int E = kSelBins / kSelThreads;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int bin = threadIdx.x * E + e;
-      const int lo = bin ? (int)st.h[bin - 1] : 0, hi = (int)st.h[bin];
-      // insertion sort of the (few) positions of the bin, then write them out
-      for (int i = lo + 1; i < hi; ++i) {
-        const int32_t v = tmp[i];
-        int j = i - 1;
-        while (j >= lo && tmp[j] > v) {
-          tmp[j + 1] = tmp[j];
-          --j;
-        }
-        tmp[j + 1] = v;
-      }
-      for (int i = lo; i < hi; ++i) out[i] = tmp[i];
-    }
-  }
+  sel_write_ordered(st, sel, ngt + kr, 0, nc, reinterpret_cast<int32_t*>(cand), out);
 }
 
 // Block maxima over candidate positions: bmax[r][b] = max score in block b.

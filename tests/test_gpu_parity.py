@@ -210,6 +210,40 @@ def test_select_all_equal_falls_back_to_exact(R, n):
         assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
 
 
+def test_select_cluster_finish_cases():
+    """Decode-sized rows on 8-CTA clusters, through the finish that ranks the
+    threshold prefix's keys on every CTA and through its fallback: the top
+    keys all in one CTA's slice; ties at the threshold under and over the
+    number of prefix keys a CTA takes (256); distinct keys that share the
+    threshold's 22-bit prefix; ties and near-ties spread over the slices."""
+    rng = np.random.default_rng(43)
+    n = 131072
+    rows = []
+    x = rng.random(n).astype(np.float32)
+    x[100:100 + 1500] += np.float32(1.0)                      # the top keys in slice 0
+    rows.append(x)
+    for nt in (200, 300):                                      # 1000 clear winners + nt ties
+        x = rng.random(n).astype(np.float32)
+        pos = rng.choice(n - 200, 1000 + nt, replace=False)
+        x[pos[:1000]] = np.float32(2.0)
+        x[pos[1000:]] = np.float32(1.5)
+        rows.append(x)
+    x = rng.random(n).astype(np.float32)                       # 100 keys sharing a 22-bit prefix
+    pos = rng.choice(n - 200, 1100, replace=False)
+    x[pos[:1000]] = np.float32(2.0)
+    bits = np.float32(1.5).view(np.uint32) + rng.permutation(100).astype(np.uint32)
+    x[pos[1000:]] = bits.view(np.float32)
+    rows.append(x)
+    x = rng.integers(0, 2000, n).astype(np.float32)            # ties spread over every slice
+    rows.append(x)
+    S = np.stack(rows)
+    ts = [n - 1] * len(rows)
+    idx, cnt = gpu_select_on(S, ts)
+    for r in range(len(rows)):
+        oi, oc = oracle.topk_select(S[r], ts[r])
+        assert int(cnt[r]) == oc and np.array_equal(idx[r], oi), r
+
+
 def test_select_large_k_exact_kernel():
     """k above the sampled kernel's limit runs the exact cluster kernel."""
     rng = np.random.default_rng(37)
