@@ -253,8 +253,7 @@ hs2_status hs2_kv_append(const hs2_problem* p, const void* K_new, const void* V_
  *     arguments must be at most 16 MiB (16,777,216 bytes); larger problems
  *     return HS2_ERR_WORKSPACE and launch nothing.
  *   - The first call on a device looks up the array's device address (a CUDA
- *     runtime query, no allocation); make that first call before any stream
- *     capture.
+ *     runtime query, no allocation).
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents.  Nothing in it needs to start at zero: every scratch entry
  *     whose value reaches idx or count was written earlier in the same call
