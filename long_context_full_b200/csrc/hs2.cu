@@ -601,13 +601,12 @@ hs2_status run_sparse(const hs2_problem* p, const void* Q_l, const void* K, cons
     // many rows (a chunk of queries): one CTA per row, no cluster
     e = launch(k_sparse_rows_bf16, dim3((unsigned)rows), dim3(32 * kSrWarps), kSrSmem, st, 0, a);
   } else if (p->dtype == HS2_BF16) {
-    CUtensorMap mk, mv;
+    CUtensorMap mk;  // K rows by TMA; V rows by cp.async
     const int64_t map_rows = p->total_kv * p->Hkv;
-    if (encode_map2(&mk, K, map_rows, kD, 1) != HS2_OK || encode_map2(&mv, V, map_rows, kD, 1) != HS2_OK)
-      return HS2_ERR_CUDA;
+    if (encode_map2(&mk, K, map_rows, kD, 1) != HS2_OK) return HS2_ERR_CUDA;
     // few rows (a small decode batch): 16 CTAs per row, half the gathers each
     const int cs = (dev->sparse16 && rows * 16 <= (int64_t)dev->sms) ? 16 : kSpCluster;
-    e = launch(k_sparse_bf16, dim3((unsigned)(rows * cs)), dim3(32 * kSpWarps), kSpGatherSmem, st, cs, mk, mv, a);
+    e = launch(k_sparse_bf16, dim3((unsigned)(rows * cs)), dim3(32 * kSpWarps), kSpGatherSmem, st, cs, mk, a);
   } else {
     const int G = a.G;
     if (G <= 1) e = launch_cluster(k_sparse_f32<1>, ctas, 32 * kSpWarps, 0, kSpCluster, st, a);

@@ -9,9 +9,10 @@
 //
 // Few rows (decode): one thread-block cluster of 8 CTAs (16 when the rows are
 // few) per (query, KV group) row.  CTA c takes the c-th share of the row's
-// index list and reads those K/V rows - bf16: TMA gather4 instructions, four
-// rows of a 2-D (position, KV head) x 128 tensor map each, in 64-column halves
-// with the 128-byte swizzle; fp32: each warp loads its rows straight into
+// index list and reads those K/V rows - bf16: K by TMA gather4 instructions,
+// four rows of a 2-D (position, KV head) x 128 tensor map each, in 64-column
+// halves with the 128-byte swizzle, and V at the same time by every thread's
+// 16-byte cp.async copies into the same layout; fp32: each warp loads its rows straight into
 // registers, 16 bytes per lane - runs an online softmax per warp (tensor cores
 // for bf16), folds its warps into one partial,
 // and the cluster merges the partials through distributed shared memory, CTA c
@@ -245,9 +246,14 @@ __device__ __forceinline__ void sparse_cluster_merge(const SparseArgs& a, int64_
 // ----------------------------------------------------------------------------
 // bf16: tensor-core S^T = K Q^T and O^T += V^T P^T per 16-key slice, the same
 // fragment scheme as the decode pass (P^T by one movmatrix transpose).
+// One arrival on ``bar`` once every cp.async this thread has issued so far has
+// landed; the barrier's expected count includes it.
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_constant__ CUtensorMap tmK,
-                                                                const __grid_constant__ CUtensorMap tmV,
                                                                 const __grid_constant__ SparseArgs a) {
   grid_dep_wait();  // the previous kernel on the stream has finished
   extern __shared__ uint8_t sp_dyn[];
@@ -258,8 +264,10 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
   cg::cluster_group cl = cg::this_cluster();
   const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
   if (threadIdx.x == 0) {
-    mbar_init(&gbar[0], 1);  // thread 0 arrives with the bytes of the group
-    mbar_init(&gbar[1], 1);
+    // thread 0 arrives with the bytes of the group's K copies, and every
+    // thread once its own V copies of the group have landed
+    mbar_init(&gbar[0], 1 + blockDim.x);
+    mbar_init(&gbar[1], 1 + blockDim.x);
     fence_mbar_init();
   }
   // the list entries of this CTA's share when the list is full (count ==
@@ -318,15 +326,17 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
       spos[row] = pos;
     }
     __syncthreads();
-    // gather: one TMA gather4 per 4 rows and per 64-column half of K and of V
-    // (rows past pn or with an invalid index load a row of the sequence that
-    // is then masked out).  Two copy groups on their own barriers: the first
-    // half of the slices is scored while the second half is still in flight.
-    // Thread 0 arrives on each group with its byte count before any copy.
+    // gather: K by TMA, one gather4 per 4 rows and per 64-column half; V by
+    // 16-byte cp.async copies of every thread into the same swizzled layout,
+    // so the TMA engine and the load/store units fetch at the same time (rows
+    // past pn or with an invalid index load a row of the sequence that is then
+    // masked out).  Two copy groups on their own barriers: the first half of
+    // the slices is scored while the second half is still in flight.  Thread 0
+    // arrives on each group with its K byte count before any copy.
     const int nA = (ntile + 1) / 2;
     if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(&gbar[0], (uint32_t)(nA * 16) * 4u * 128u);
-      mbar_arrive_expect_tx(&gbar[1], (uint32_t)((ntile - nA) * 16) * 4u * 128u);
+      mbar_arrive_expect_tx(&gbar[0], (uint32_t)(nA * 16) * 2u * 128u);
+      mbar_arrive_expect_tx(&gbar[1], (uint32_t)((ntile - nA) * 16) * 2u * 128u);
     }
     __syncthreads();
     for (int q = threadIdx.x; q < ntile * 4; q += blockDim.x) {
@@ -343,8 +353,21 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
       const uint32_t off = (uint32_t)row0 * 128u;
       tma_gather4(sK + off, &tmK, bar, 0, rr[0], rr[1], rr[2], rr[3]);
       tma_gather4(sK + kSpHalfBytes + off, &tmK, bar, 64, rr[0], rr[1], rr[2], rr[3]);
-      tma_gather4(sV + off, &tmV, bar, 0, rr[0], rr[1], rr[2], rr[3]);
-      tma_gather4(sV + kSpHalfBytes + off, &tmV, bar, 64, rr[0], rr[1], rr[2], rr[3]);
+    }
+    {
+      const bf16* Vg = static_cast<const bf16*>(a.V);
+      for (int grp = 0; grp < 2; ++grp) {
+        const int c0 = (grp == 0 ? 0 : nA * 16) * 16, c1 = (grp == 0 ? nA * 16 : ntile * 16) * 16;
+        for (int j = c0 + (int)threadIdx.x; j < c1; j += blockDim.x) {  // 16 chunks of 16 B a row
+          const int row = j >> 4, half = (j >> 3) & 1, chunk = j & 7;
+          const int64_t pos = spos[row];
+          int64_t mr = (s.kv_start + (pos >= 0 ? pos : 0)) * a.Hkv + s.g;
+          mr = mr < 0 ? 0 : (mr >= map_rows ? map_rows - 1 : mr);
+          cp_async16(sV + half * kSpHalfBytes + row * 128 + ((chunk ^ (row & 7)) << 4),
+                     Vg + mr * kD + half * 64 + chunk * 8, 16);
+        }
+        cp_async_mbar_arrive_noinc(&gbar[grp]);
+      }
     }
     for (int half = 0; half < 2; ++half) {
       if (!mbar_wait(&gbar[half], (uint32_t)(piece & 1))) record_error(a.err, HS2_ERR_TIMEOUT);
@@ -400,6 +423,7 @@ __global__ void __launch_bounds__(32 * kSpWarps) k_sparse_bf16(const __grid_cons
     __syncthreads();  // the next piece overwrites the staged rows
     fence_proxy_async_smem();  // ... by TMA copies after these reads
   }
+  cp_async_wait_all();  // (after a timed-out wait) no copy lands after the CTA is gone
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, off);
