@@ -544,10 +544,11 @@ __global__ void __launch_bounds__(kCombThreads) k_decode_combine(const __grid_co
 //      c, c + P*Hkv, ... into O, as k_decode_combine does;
 //   2. for each piece: the final (m_h, l_h) of the group's G heads, from the
 //      partials (lane-parallel, one warp per head) or from ml_in;
-//   3. score two keys per thread per stage, the writes coalesced along j.
+//   3. score kFinChunk / 256 keys per thread per stage, the writes coalesced
+//      along j.
 // ----------------------------------------------------------------------------
-constexpr int kFinChunk = 512;
-constexpr int kFinStages = 4;
+constexpr int kFinChunk = 1024;
+constexpr int kFinStages = 3;
 constexpr int kFinWarps = 8;
 constexpr int kFinThreads = 32 * (kFinWarps + 1);
 constexpr float kLog2e = 1.4426950408889634f;
