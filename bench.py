@@ -250,21 +250,21 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(w, budget_s: float = 12.0):
-    """Oracle throughput in query-tok/s on whole (query, KV group) units until
+    """Oracle throughput in query-tok/s on whole (query, KV group) units, the
+    batch's units in turn (again from the first when all are done) until
     ``budget_s`` of CPU time has been spent (at least one unit)."""
+    n = w.q.shape[0] * w.Hkv
     units, t0 = 0, time.perf_counter()
-    for r in range(w.q.shape[0]):
-        for g in range(w.Hkv):
-            oracle_unit(w, r, g)
-            units += 1
-            if time.perf_counter() - t0 > budget_s:
-                break
+    while True:
+        r, g = divmod(units % n, w.Hkv)
+        oracle_unit(w, r, g)
+        units += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
     return {"value": (units / w.Hkv) / dt, "unit": UNIT, "cores": blas_threads(),
             "kind": "oracle",
-            "sample": f"{units} (query, KV-group) units of {w.q.shape[0] * w.Hkv}: full attention "
+            "sample": f"{units} (query, KV-group) units, the batch's {n} in turn: full attention "
                       f"of the group's {w.Hq // w.Hkv} heads over {int(w.kv_lens[0])} keys, scores, top-k "
                       f"select, {w.n_layers} sparse layers; float64 numpy, {dt:.1f} s"}
 
