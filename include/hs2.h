@@ -126,6 +126,12 @@ typedef struct {
  * Returns HS2_OK, or INVALID_ARG / UNSUPPORTED / WORKSPACE / CUDA.
  */
 hs2_status hs2_full_attn_workspace_size(const hs2_problem* p, size_t* bytes);
+/* The number of kernels one hs2_full_attn_scores call launches for ``p`` on
+ * the current device (*n = 0 when total_q = 0): decode 2 (the pass, then the
+ * O merge and score finalize); bf16 chunks 1, or 3 when the visible keys are
+ * split over several CTAs per query tile (statistics, then scores and O
+ * shares, then the O sum); float32 chunks 2.  Returns HS2_OK or INVALID_ARG. */
+hs2_status hs2_full_attn_launches(const hs2_problem* p, int32_t* n);
 hs2_status hs2_full_attn_scores(const hs2_problem* p, const void* Q, const void* K,
                                 const void* V, void* O, float* scores, int64_t score_stride,
                                 void* workspace, size_t workspace_bytes, void* stream);

@@ -108,8 +108,6 @@ class HybridBlockStep:
 
     def launches_per_step(self) -> int:
         """Kernels one ``run`` launches."""
-        # decode: split pass, then O merge + scores; chunk: one tcgen05 kernel
-        # (bf16) or attention + score kernels (fp32)
-        full = 2 if self.max_q <= 1 else (1 if self.dtype == torch.bfloat16 else 2)
+        full = hs2.hs2_full_attn_launches(self.problem)
         sel = 1 if self.select == "token" else 3
         return full + sel + self.n_layers

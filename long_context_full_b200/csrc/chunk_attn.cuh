@@ -32,9 +32,15 @@ struct ChunkArgs {
   float* scores;
   int64_t stride;
   int* err;
+  // tensor-core kernel, visible keys split over ksplit CTAs per query tile
+  // (ksplit = 1: both passes in one CTA, O written directly):
+  int ksplit;             // CTAs per query tile; blockIdx.z = sequence * ksplit + split
+  int mode;               // 0: both passes; 1: statistics only; 2: scores and O only
+  float* part_ml;         // [ksplit][total_q * Hq][2] each split's (max in base 2, sum)
+  float* part_o;          // [ksplit][total_q * Hq][D] each split's share of O
 };
 
-// Sequence-level geometry of CTA (blockIdx.x = query tile, blockIdx.z = sequence).
+// Sequence-level geometry of CTA (blockIdx.x = query tile, sequence b).
 struct ChTile {
   int64_t q0;       // first query row (packed index) of the tile
   int nq;           // query tokens in the tile
@@ -42,8 +48,7 @@ struct ChTile {
   int64_t N;        // keys of the sequence
   int64_t t0;       // position of the tile's first query
 };
-__device__ __forceinline__ bool chunk_tile(const ChunkArgs& a, ChTile& c) {
-  const int b = blockIdx.z;
+__device__ __forceinline__ bool chunk_tile(const ChunkArgs& a, int b, ChTile& c) {
   const int64_t qs = __ldg(a.qoff + b), qe = __ldg(a.qoff + b + 1);
   c.kv0 = __ldg(a.kvoff + b);
   c.N = __ldg(a.kvoff + b + 1) - c.kv0;

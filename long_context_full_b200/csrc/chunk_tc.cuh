@@ -28,6 +28,15 @@
 // buffers (tile t, buffer b) at 256t + 128b; pass B, S_t/P_t at 128t and O_t
 // at 256 + 128t.  S_t of the next key tile is issued right after the
 // O_t += P_t V that reads P_t: tcgen05.mma from one thread execute in order.
+//
+// Key split (a.ksplit > 1): the query tiles alone leave the last wave of CTAs
+// part-empty (256 tiles on 148 SMs run in 2 waves, the second 73 % full), so
+// the visible key tiles are cut into ksplit contiguous ranges, one CTA each,
+// in two launches: mode 1 runs pass A over its range and writes each row's
+// (max, sum); mode 2 merges the ranges' (max, sum) into the row's exact
+// statistics, runs pass B over its range (P is then exact, so the scores of its
+// keys are final and its share of O needs no rescaling) and writes that share
+// in float32; k_chunk_o_sum adds the shares in a fixed order.
 #pragma once
 
 #include <type_traits>
@@ -65,8 +74,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t sb_full[2], pb_full[2], o_full;  // pass B: [Q tile]
   __shared__ uint32_t tmem_base_sh;
 
+  const int ks = a.ksplit > 0 ? a.ksplit : 1;
+  const int split = (int)blockIdx.z % ks;
   ChTile c;
-  if (!chunk_tile(a, c)) return;
+  if (!chunk_tile(a, (int)blockIdx.z / ks, c)) return;
+  const bool doA = a.mode != 2, doB = a.mode != 1;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
   uint8_t* sK = base + kTcQTiles * kTcQBytes;
@@ -74,7 +86,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
   const int64_t nkeys = c.t0 + c.nq;  // keys [0, t_last] are visible to some row
-  const int n = (int)((nkeys + kTcKeys - 1) / kTcKeys);
+  const int ntot = (int)((nkeys + kTcKeys - 1) / kTcKeys);
+  // this CTA's key tiles [j0, j0 + n)
+  const int j0 = (int)((int64_t)ntot * split / ks);
+  const int n = (int)((int64_t)ntot * (split + 1) / ks) - j0;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
@@ -130,13 +145,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return true;
       };
       int kf = 0, vf = 0;
-      for (int j = 0; j < n && ok; ++j) {
-        if ((ok = fill(k_full, k_empty, sK, kTcKStages, &tmK, kf, j))) ++kf;
+      for (int j = 0; j < n && ok && doA; ++j) {
+        if ((ok = fill(k_full, k_empty, sK, kTcKStages, &tmK, kf, j0 + j))) ++kf;
       }
-      for (int j = 0; j < n && ok; ++j) {
-        if (!(ok = fill(k_full, k_empty, sK, kTcKStages, &tmK, kf, j))) break;
+      for (int j = 0; j < n && ok && doB; ++j) {
+        if (!(ok = fill(k_full, k_empty, sK, kTcKStages, &tmK, kf, j0 + j))) break;
         ++kf;
-        if (!(ok = fill(v_full, v_empty, sV, kTcVStages, &tmV, vf, j))) break;
+        if (!(ok = fill(v_full, v_empty, sV, kTcVStages, &tmV, vf, j0 + j))) break;
         ++vf;
       }
       if (!ok) record_error(a.err, HS2_ERR_TIMEOUT);
@@ -175,8 +190,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       };
       auto kwait = [&](int f) { return mbar_wait(&k_full[f % kTcKStages], (uint32_t)(f / kTcKStages) & 1u); };
-      // ---- pass A
-      for (int j = 0; j < n && ok; ++j) {
+      // ---- pass A (local tile j = key tile j0 + j)
+      for (int j = 0; j < n && ok && doA; ++j) {
         if (!(ok = kwait(j))) break;
         const int b = j & 1;
         for (int t = 0; t < 2 && ok; ++t) {
@@ -188,23 +203,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma_commit(&k_empty[j % kTcKStages]);
       }
       // every S buffer of pass A has been read before pass B reuses the columns
-      for (int j = (n > 2 ? n - 2 : 0); j < n && ok; ++j)
+      for (int j = (n > 2 ? n - 2 : 0); j < n && ok && doA; ++j)
         for (int t = 0; t < 2 && ok; ++t) ok = mbar_wait(&sa_free[t][j & 1], (uint32_t)(j >> 1) & 1u);
       tc_fence_after();
-      // ---- pass B
-      if (ok && n > 0 && (ok = kwait(n))) {
+      // ---- pass B (its K fills follow pass A's)
+      const int kb = doA ? n : 0;
+      if (doB && ok && n > 0 && (ok = kwait(kb))) {
         tc_fence_after();
-        mma_s(0, 0, n % kTcKStages);
+        mma_s(0, 0, kb % kTcKStages);
         umma_commit(&sb_full[0]);
-        mma_s(128, 1, n % kTcKStages);
+        mma_s(128, 1, kb % kTcKStages);
         umma_commit(&sb_full[1]);
-        umma_commit(&k_empty[n % kTcKStages]);
+        umma_commit(&k_empty[kb % kTcKStages]);
       }
-      for (int j = 0; j < n && ok; ++j) {
+      for (int j = 0; j < n && ok && doB; ++j) {
         const int vst = j % kTcVStages;
         if (!(ok = mbar_wait(&v_full[vst], (uint32_t)(j / kTcVStages) & 1u))) break;
         const uint64_t vd = umma_desc_sw128(smem_u32(sV + vst * kTcTileBytes), kTcTileBytes / 2, 1024);
-        const int kf = n + j + 1;  // the K fill of key tile j + 1
+        const int kf = kb + j + 1;  // the K fill of local tile j + 1
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = mbar_wait(&pb_full[t], (uint32_t)j & 1u))) break;
           tc_fence_after();
@@ -249,7 +265,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // ---- pass A: running max and sum
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < n && doA; ++j) {
       const int b = j & 1;
       if (ok && !mbar_wait(&sa_full[tq][b], (uint32_t)(j >> 1) & 1u)) {
         record_error(a.err, HS2_ERR_TIMEOUT);
@@ -259,7 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       if (ok) {
         // the whole 128-key row of S at once: one wait, 128-wide independent work
-        const int64_t k0 = (int64_t)j * kTcKeys;
+        const int64_t k0 = (int64_t)(j0 + j) * kTcKeys;
         uint32_t r[4][32];
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_ld32(trow + 256 * tq + 128 * b + 32 * q, r[q]);
@@ -299,16 +315,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sa_free[tq][b]);
     }
+    const int64_t nrows = a.total_q * a.Hq;
+    if (a.mode == 1) {  // statistics of this key range only (m = -inf, l = 0 if it has none)
+      if (rv) {
+        a.part_ml[((int64_t)split * nrows + hrow) * 2] = m;
+        a.part_ml[((int64_t)split * nrows + hrow) * 2 + 1] = l;
+      }
+    }
+    if (a.mode == 2 && rv) {  // the row's statistics over all ranges, in range order
+      float M = -INFINITY;
+      for (int q = 0; q < ks; ++q) M = fmaxf(M, a.part_ml[((int64_t)q * nrows + hrow) * 2]);
+      float L = 0.f;
+      for (int q = 0; q < ks; ++q) {
+        const float mq = a.part_ml[((int64_t)q * nrows + hrow) * 2];
+        if (mq != -INFINITY) L += a.part_ml[((int64_t)q * nrows + hrow) * 2 + 1] * exp2f(mq - M);
+      }
+      m = M;
+      l = L;
+    }
     const float mb = (rv && l > 0.f) ? m + log2f(l) : 0.f;  // l >= 1 for a visible row
     // ---- pass B: P (handed to the MMA warp first), then the scores
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < n && doB; ++j) {
       if (ok && !mbar_wait(&sb_full[tq], (uint32_t)j & 1u)) {
         record_error(a.err, HS2_ERR_TIMEOUT);
         ok = false;
       }
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      const int64_t k0 = (int64_t)j * kTcKeys;
+      const int64_t k0 = (int64_t)(j0 + j) * kTcKeys;
       const bool full = all_rv && k0 + kTcKeys - 1 <= t_min;  // no key of the tile is masked
       // keys k0 .. k0+nv-1 are visible to this row
       const int nv = full ? kTcKeys : (rv ? (int)max((int64_t)0, min((int64_t)kTcKeys, t - k0 + 1)) : 0);
@@ -381,7 +415,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
-    // ---- O of this row: bf16 out of tensor memory
+    // ---- O of this row: bf16 out of tensor memory (mode 2: this range's
+    // float32 share, zero for a range with no key tile)
     if (ok && !mbar_wait(&o_full, 0)) {
       record_error(a.err, HS2_ERR_TIMEOUT);
       ok = false;
@@ -390,7 +425,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     bf16* O = static_cast<bf16*>(a.O);
 #pragma unroll 1
-    for (int ch = 0; ch < 4 && ok; ++ch) {
+    for (int ch = 0; ch < 4 && ok && a.mode == 2; ++ch) {
+      uint32_t r[32];
+      if (n > 0) {
+        tmem_ld32(trow + 256 + 128 * tq + ch * 32, r);
+        tmem_wait_ld();
+      }
+      if (rv) {
+        float4* dst = reinterpret_cast<float4*>(a.part_o + ((int64_t)split * nrows + hrow) * kD + ch * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = n > 0 ? make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                       __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll 1
+    for (int ch = 0; ch < 4 && ok && a.mode == 0; ++ch) {
       uint32_t r[32];
       tmem_ld32(trow + 256 + 128 * tq + ch * 32, r);
       tmem_wait_ld();
@@ -410,6 +461,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// O of a key-split chunk: the ranges' float32 shares added in range order,
+// written as bf16.  One thread per 4 columns of a row.
+__global__ void __launch_bounds__(256) k_chunk_o_sum(const float* part_o, int ks, int64_t nrows, bf16* O) {
+  grid_dep_wait();  // the previous kernel on the stream has finished
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // float4 index
+  if (i >= nrows * (kD / 4)) return;
+  float4 acc = reinterpret_cast<const float4*>(part_o)[i];
+  for (int q = 1; q < ks; ++q) {
+    const float4 v = reinterpret_cast<const float4*>(part_o)[(int64_t)q * nrows * (kD / 4) + i];
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  uint2 pk;
+  pk.x = pack_bf16(acc.x, acc.y);
+  pk.y = pack_bf16(acc.z, acc.w);
+  reinterpret_cast<uint2*>(O)[i] = pk;
 }
 
 }  // namespace hs2

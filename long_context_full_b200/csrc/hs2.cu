@@ -323,13 +323,44 @@ hs2_status run_decode(const hs2_problem* p, const DeviceInfo& dev, const void* Q
 // --------------------------------------------------------------------------
 struct ChunkPlan {
   float* ml;
+  int ks;          // key ranges per query tile of the tensor-core kernel
+  float* part_ml;  // ks > 1: each range's row statistics
+  float* part_o;   // ks > 1: each range's share of O (float32)
   size_t bytes;
 };
 
-ChunkPlan plan_chunk(const hs2_problem* p, const DeviceInfo&, void* ws) {
+// Key ranges per query tile of the tensor-core chunk kernel (one CTA per SM):
+// the count in 1 .. 8 that runs the CTAs in the fewest waves per unit of work
+// (the smallest on a tie), each range keeping at least 8 key tiles of the
+// longest sequence.
+int chunk_ksplit(const hs2_problem* p, const DeviceInfo& dev) {
+  if (p->dtype != HS2_BF16 || dev.sms <= 0) return 1;
+  const int64_t G = p->Hq / p->Hkv;
+  const int64_t QT = kTcQTiles * kTcRows / G;
+  const int64_t units = (p->max_q_len + QT - 1) / QT * p->Hkv * p->B;
+  const int64_t tiles = (p->max_kv_len + kTcKeys - 1) / kTcKeys;
+  int best = 1;
+  int64_t best_waves = (units + dev.sms - 1) / dev.sms;  // for ks = 1
+  for (int k = 2; k <= 8; ++k) {
+    if (tiles < 8 * (int64_t)k || (int64_t)p->B * k > 65535) break;
+    const int64_t waves = (units * k + dev.sms - 1) / dev.sms;
+    if (waves * best < best_waves * k) {  // waves / k < best_waves / best
+      best = k;
+      best_waves = waves;
+    }
+  }
+  return best;
+}
+
+ChunkPlan plan_chunk(const hs2_problem* p, const DeviceInfo& dev, void* ws) {
   ChunkPlan c{};
   Carve w(ws);
   c.ml = w.take<float>((size_t)p->total_q * p->Hq * 2);
+  c.ks = chunk_ksplit(p, dev);
+  if (c.ks > 1) {
+    c.part_ml = w.take<float>((size_t)c.ks * p->total_q * p->Hq * 2);
+    c.part_o = w.take<float>((size_t)c.ks * p->total_q * p->Hq * kD);
+  }
   c.bytes = w.used;
   return c;
 }
@@ -372,12 +403,28 @@ hs2_status run_chunk(const hs2_problem* p, const DeviceInfo& dev, const void* Q,
         encode_map3(&mk, K, p->total_kv, p->Hkv, 1, kTcKeys) != HS2_OK ||
         encode_map3(&mv, V, p->total_kv, p->Hkv, 1, kTcKeys) != HS2_OK)
       return HS2_ERR_CUDA;
-    const dim3 grid((unsigned)((p->max_q_len + a.QT - 1) / a.QT), p->Hkv, p->B);
-    switch (a.G) {
-      case 1: launch_chunk_tc<1>(grid, st, mq, mk, mv, a); break;
-      case 2: launch_chunk_tc<2>(grid, st, mq, mk, mv, a); break;
-      case 4: launch_chunk_tc<4>(grid, st, mq, mk, mv, a); break;
-      default: launch_chunk_tc<8>(grid, st, mq, mk, mv, a); break;
+    a.ksplit = pl.ks;
+    a.part_ml = pl.part_ml;
+    a.part_o = pl.part_o;
+    const dim3 grid((unsigned)((p->max_q_len + a.QT - 1) / a.QT), p->Hkv, (unsigned)(p->B * pl.ks));
+    auto run = [&](int mode) {
+      a.mode = mode;
+      switch (a.G) {
+        case 1: launch_chunk_tc<1>(grid, st, mq, mk, mv, a); break;
+        case 2: launch_chunk_tc<2>(grid, st, mq, mk, mv, a); break;
+        case 4: launch_chunk_tc<4>(grid, st, mq, mk, mv, a); break;
+        default: launch_chunk_tc<8>(grid, st, mq, mk, mv, a); break;
+      }
+    };
+    if (pl.ks == 1) {
+      run(0);
+    } else {  // statistics per key range, then scores and O shares, then O
+      run(1);
+      run(2);
+      const int64_t nrows = p->total_q * p->Hq;
+      const int64_t n4 = nrows * (kD / 4);
+      launch(k_chunk_o_sum, dim3((unsigned)((n4 + 255) / 256)), dim3(256), 0, st, 0,
+             (const float*)pl.part_o, pl.ks, nrows, static_cast<bf16*>(O));
     }
     return launch_status();
   }
@@ -461,6 +508,19 @@ hs2_status hs2_full_attn_workspace_size(const hs2_problem* p, size_t* bytes) {
   if ((s = device_info(&dev)) != HS2_OK) return s;
   if (p->max_q_len <= 1) *bytes = plan_decode(p, *dev, nullptr).bytes;
   else *bytes = plan_chunk(p, *dev, nullptr).bytes;
+  return HS2_OK;
+}
+
+hs2_status hs2_full_attn_launches(const hs2_problem* p, int32_t* n) {
+  if (!n) return HS2_ERR_INVALID_ARG;
+  hs2_status s = check_problem(p);
+  if (s != HS2_OK) return s;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != HS2_OK) return s;
+  if (p->total_q == 0) *n = 0;
+  else if (p->max_q_len <= 1) *n = 2;
+  else if (p->dtype == HS2_BF16) *n = chunk_ksplit(p, *dev) > 1 ? 3 : 1;
+  else *n = 2;
   return HS2_OK;
 }
 

@@ -29,7 +29,7 @@ HS2_F32 = 0
 HS2_BF16 = 1
 
 EXPORTED = [
-    "hs2_full_attn_workspace_size", "hs2_full_attn_scores",
+    "hs2_full_attn_workspace_size", "hs2_full_attn_launches", "hs2_full_attn_scores",
     "hs2_topk_workspace_size", "hs2_topk_select",
     "hs2_block_select_workspace_size", "hs2_block_select", "hs2_block_select_noalloc",
     "hs2_sparse_attn_workspace_size", "hs2_sparse_attn", "hs2_kv_append", "hs2_swa_attn",
@@ -75,6 +75,7 @@ def load() -> ctypes.CDLL:
     psz = ctypes.POINTER(ctypes.c_size_t)
     sig = {
         "hs2_full_attn_workspace_size": [P, psz],
+        "hs2_full_attn_launches": [P, ctypes.POINTER(i32)],
         "hs2_full_attn_scores": [P, vp, vp, vp, vp, vp, i64, vp, sz, vp],
         "hs2_topk_workspace_size": [P, i32, i32, psz],
         "hs2_topk_select": [P, vp, i64, i32, i32, vp, vp, vp, sz, vp],
@@ -168,6 +169,12 @@ def _ws(workspace):
 
 def hs2_full_attn_workspace_size(p: Problem) -> int:
     return _size(load().hs2_full_attn_workspace_size, ctypes.byref(p))
+
+
+def hs2_full_attn_launches(p: Problem) -> int:
+    n = ctypes.c_int32(0)
+    _check(load().hs2_full_attn_launches(ctypes.byref(p), ctypes.byref(n)), "hs2_full_attn_launches")
+    return int(n.value)
 
 
 def hs2_full_attn_scores(p: Problem, Q, K, V, O, scores, score_stride, workspace, stream=None):
