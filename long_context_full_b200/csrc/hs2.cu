@@ -331,8 +331,9 @@ struct ChunkPlan {
 
 // Key ranges per query tile of the tensor-core chunk kernel (one CTA per SM):
 // the count in 1 .. 8 that runs the CTAs in the fewest waves per unit of work
-// (the smallest on a tie), each range keeping at least 8 key tiles of the
-// longest sequence.
+// (the smallest on a tie), each range keeping at least 64 key tiles (8192 keys)
+// of the longest sequence: with 36 tiles a range (a 16K-key context) the two
+// launches and the O shares cost more than the fuller waves win.
 int chunk_ksplit(const hs2_problem* p, const DeviceInfo& dev) {
   if (p->dtype != HS2_BF16 || dev.sms <= 0) return 1;
   const int64_t G = p->Hq / p->Hkv;
@@ -342,7 +343,7 @@ int chunk_ksplit(const hs2_problem* p, const DeviceInfo& dev) {
   int best = 1;
   int64_t best_waves = (units + dev.sms - 1) / dev.sms;  // for ks = 1
   for (int k = 2; k <= 8; ++k) {
-    if (tiles < 8 * (int64_t)k || (int64_t)p->B * k > 65535) break;
+    if (tiles < 64 * (int64_t)k || (int64_t)p->B * k > 65535) break;
     const int64_t waves = (units * k + dev.sms - 1) / dev.sms;
     if (waves * best < best_waves * k) {  // waves / k < best_waves / best
       best = k;

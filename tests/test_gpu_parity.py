@@ -297,6 +297,19 @@ def test_chunk_causal(dtype):
     full_check(w)
 
 
+def test_chunk_key_split_bf16():
+    """A chunk whose query tiles alone would leave most SMs idle: the visible
+    keys of each tile are split over several CTAs (statistics per range, then
+    scores and O shares per range, then the O sum), with a second, short
+    sequence whose ranges are a few key tiles each."""
+    w = synth.make_workload("chunks", 63, "bf16", 32, 4, 128, [20000, 3000], [64, 40], 1)
+    p = hs2.make_problem(w.B, w.Hq, w.Hkv, w.D, hs2.HS2_BF16, torch.from_numpy(w.q_offsets).cuda(),
+                         torch.from_numpy(w.kv_offsets).cuda(), int(w.q_lens.sum()),
+                         int(w.kv_lens.sum()), int(w.q_lens.max()), int(w.kv_lens.max()), w.scale)
+    assert hs2.hs2_full_attn_launches(p) == 3  # the split form runs on this shape
+    full_check(w)
+
+
 def test_chunk_gqa_bf16():
     for Hq, Hkv in ((4, 4), (8, 4), (8, 2), (32, 4)):
         w = synth.make_workload("chunkg", 62, "bf16", Hq, Hkv, 128, [2500], [150], 1)
