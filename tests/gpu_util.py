@@ -39,7 +39,7 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy().astype(np.float64)
 
 
-class GpuRun:
+class CudaPathRun:
     """The CUDA path on one workload: full attention + scores, selection, sparse layers."""
 
     def __init__(self, w: synth.Workload, select: str = "token"):

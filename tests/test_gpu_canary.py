@@ -20,7 +20,7 @@ import torch
 
 import synth
 from long_context_full_b200 import hs2
-from tests.gpu_util import GpuRun, OracleRows, check_O, check_scores, to_f64
+from tests.gpu_util import CudaPathRun, OracleRows, check_O, check_scores, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -70,7 +70,7 @@ CASES = {
 def test_outputs_stay_in_bounds(case, pad):
     dtype, Hq, Hkv, kv_lens, q_lens = CASES[case]
     w = synth.make_workload("can_" + case, 97, dtype, Hq, Hkv, 128, kv_lens, q_lens, 1)
-    ref = GpuRun(w)
+    ref = CudaPathRun(w)
     out = ref.run()
     step = ref.step
     p = step.problem

@@ -9,7 +9,7 @@ import torch
 
 import synth
 from long_context_full_b200 import hs2
-from tests.gpu_util import GpuRun
+from tests.gpu_util import CudaPathRun
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +29,7 @@ def _same_scores(a, b, tpos):
 def test_inconsistent_kv_offsets_are_reported(bad):
     w = synth.make_workload("devin", 41, "bf16", 8, 2, 128, [2000, 1000], [1, 1], 1)
     tpos = np.repeat(w.query_positions(), w.Hkv)
-    run = GpuRun(w)
+    run = CudaPathRun(w)
     clean = _outputs(run.run())
     good = run.step.kv_offsets.clone()
 
@@ -45,7 +45,7 @@ def test_inconsistent_kv_offsets_are_reported(bad):
         assert _same_scores(out["scores"][:G], clean["scores"][:G], tpos[:G])
 
     run.step.kv_offsets.copy_(good)
-    again = _outputs(run.run())  # GpuRun.run asserts HS2_OK
+    again = _outputs(run.run())  # CudaPathRun.run asserts HS2_OK
     for name in ("O", "idx", "count", "O1"):
         assert torch.equal(again[name], clean[name]), name
     assert _same_scores(again["scores"], clean["scores"], tpos)

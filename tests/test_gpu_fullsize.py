@@ -7,14 +7,14 @@ import pytest
 
 import oracle
 import synth
-from tests.gpu_util import (GpuRun, OracleRows, check_O, check_block_sets, check_index_sets,
+from tests.gpu_util import (CudaPathRun, OracleRows, check_O, check_block_sets, check_index_sets,
                             check_scores, gpu_select_on, to_f64)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
 def check_rows(w, rows, select="token"):
-    run = GpuRun(w, select)
+    run = CudaPathRun(w, select)
     out = run.run()
     ora = OracleRows(w)
     Og = to_f64(out.O)

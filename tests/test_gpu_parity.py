@@ -7,7 +7,7 @@ import torch
 import oracle
 import synth
 from long_context_full_b200 import hs2
-from tests.gpu_util import (GpuRun, OracleRows, check_O, check_block_sets, check_index_sets,
+from tests.gpu_util import (CudaPathRun, OracleRows, check_O, check_block_sets, check_index_sets,
                             check_scores, gpu_select_on, to_f64)
 
 pytestmark = pytest.mark.gpu
@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 def full_check(w, select="token", rows=None, layers=True):
     """Runs the CUDA path and checks O, scores, selection and sparse layers for
     the listed query rows (all by default).  Returns a summary dict."""
-    run = GpuRun(w, select)
+    run = CudaPathRun(w, select)
     out = run.run()
     ora = OracleRows(w)
     O = out.O
@@ -69,7 +69,7 @@ def test_sparse_equals_full_when_budget_covers_context():
     for dtype in ("f32", "bf16"):
         w = synth.make_workload("short", 11, dtype, 8, 2, 128, [1152, 700, 1], [1, 1, 1], 1)
         w.q_layers[0][:] = w.q  # same queries as the full-attention layer
-        run = GpuRun(w)
+        run = CudaPathRun(w)
         out = run.run()
         cnt = out.count.cpu().numpy()
         assert list(cnt) == [1152, 1152, 700, 700, 1, 1]
@@ -318,7 +318,7 @@ def test_chunk_gqa_bf16():
 
 def test_repeatable():
     w = synth.make_workload("rep", 71, "bf16", 32, 4, 128, [50000, 20000], [1, 1], 1)
-    run = GpuRun(w)
+    run = CudaPathRun(w)
     a = run.run()
     i1, s1, o1 = a.idx.clone(), a.scores.clone(), a.O_layers[0].clone()
     b = run.run()
@@ -327,7 +327,7 @@ def test_repeatable():
 
 def test_device_input_errors_are_reported():
     w = synth.make_workload("err", 81, "bf16", 8, 1, 128, [500], [1], 1)
-    run = GpuRun(w)
+    run = CudaPathRun(w)
     run.run()
     bad = run.step.idx.clone()
     bad[0, 3] = 600  # beyond the query position
@@ -340,7 +340,7 @@ def test_device_input_errors_are_reported():
 
 def test_host_checks_launch_nothing():
     w = synth.make_workload("chk", 91, "bf16", 8, 1, 128, [500], [1], 1)
-    run = GpuRun(w, select="block")
+    run = CudaPathRun(w, select="block")
     before = run.step.idx.clone()
     with pytest.raises(hs2.HS2Error) as e:
         hs2.hs2_block_select(run.step.problem, run.step.scores, run.step.stride, 16, 64, 128,
@@ -364,7 +364,7 @@ def test_sequences_without_queries(dtype, q_lens):
     assert summ["flips"] == 0
     summ, out = full_check(w, select="block")
     # the no-allocation block selection gives the same result on the same scores
-    run = GpuRun(w, select="block")
+    run = CudaPathRun(w, select="block")
     o = run.run()
     idx2 = torch.full_like(o.idx, 7777)
     cnt2 = torch.full_like(o.count, 7777)
